@@ -1,0 +1,519 @@
+"""Benchmark of the truly-sparse layer's hot path on B200.
+
+Workload: the single FC layer W 4096 x 4096 at 95% sparsity (838,861 nnz, uniform positions),
+bf16 values and activations with fp32 accumulation, batch N in {1, 8, 32}.  One step = the
+forward SpMM, the transposed SpMM (input gradient) and the SDDMM (weight gradient) at each of
+the three batch sizes: 9 launches.  The format build and one restructure pass are timed
+separately and reported under "preprocess" (their cost is reported, not hidden).
+
+Metric: achieved HBM GB/s under the algorithmic byte model (values + indices + row/col
+pointers + the dense operands read once + outputs written once) and useful GFLOP/s
+(2 nnz N per op).  L2 is kept cold by rotating over R independent copies of every operand
+(layout, values, activations, outputs) whose total exceeds 3x the L2 size; each step runs on
+the next copy.  Timing: CUDA events on the launching stream around K replays of CUDA graphs
+(one graph per copy, one step each), synchronised on both sides; max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (plain fp64 loops, one thread) on the same workload,
+each step a bounded sample of rows.  Under torchrun only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SpMM HBM GB/s (frac. of peak) & useful GFLOP/s=2·nnz·N at 90–99% sparsity"
+WORKLOAD = "fc-4096x4096-s95-bf16"
+BATCHES = (1, 8, 32)
+OPS = ("forward", "backward_input", "backward_weight")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- byte / flop model
+
+def op_bytes(op: str, M: int, K: int, nnz: int, N: int, s: int) -> int:
+    """Algorithmic bytes of one op: compulsory traffic, int32 indices, dense operands once."""
+    if op == "forward":
+        return nnz * (s + 4) + 4 * (M + 1) + K * N * s + M * N * s
+    if op == "backward_input":
+        return nnz * (s + 4 + 4) + 4 * (K + 1) + M * N * s + K * N * s
+    if op == "backward_weight":
+        return nnz * (4 + s) + 4 * (M + 1) + K * N * s + M * N * s
+    raise ValueError(op)
+
+
+def op_flops(nnz: int, N: int) -> int:
+    return 2 * nnz * N
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured", "sm_max_mhz": p.get("sm_max_mhz")}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback", "sm_max_mhz": 1965.0}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- our implementation
+
+def run_ours(args, rank: int, world: int, local: int) -> dict:
+    import torch
+
+    from sparse_spmm_b200 import build as build_mod
+    from sparse_spmm_b200 import snk
+    from sparse_spmm_b200 import workloads as wl
+
+    build_mod.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2**20))
+
+    layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
+    M, K, nnz = layer.M, layer.K, layer.nnz
+    s = 2
+    batches = [int(b) for b in args.batches.split(",")]
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    row_h, col_h, val_h = layer.row, layer.col, layer.values
+    xs = {N: wl.activations(K, N, "bf16", args.seed, stream=2) for N in batches}
+    dys = {N: wl.activations(M, N, "bf16", args.seed, stream=3) for N in batches}
+
+    # hot bytes of one copy: format arrays read by the products + values + activations + outputs
+    hot = nnz * (4 + 4 + 4 + s + s) + 8 * (M + K) + sum((K + M) * N * s * 2 for N in batches)
+    R = max(2, int(np.ceil(3.0 * l2 / hot)))
+    if args.rotate:
+        R = args.rotate
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    # build R copies (timing the build of the first)
+    copies = []
+    t_build = None
+    for i in range(R):
+        row, col, val = torch.from_numpy(row_h).to(dev), torch.from_numpy(col_h).to(dev), dev_bf16(val_h)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t0 = time.perf_counter()
+            L = snk.Layout(M, K, row, col, val, num_parts=args.parts)
+            t1 = time.perf_counter()
+        if i == 0:
+            t_build = t1 - t0
+        c = {"L": L}
+        for N in batches:
+            c[("X", N)] = dev_bf16(xs[N])
+            c[("dY", N)] = dev_bf16(dys[N])
+            c[("Y", N)] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            c[("dX", N)] = torch.empty((K, N), dtype=torch.bfloat16, device=dev)
+            c[("dW", N)] = torch.empty(nnz, dtype=torch.bfloat16, device=dev)
+        copies.append(c)
+    P = copies[0]["L"].num_parts
+    torch.cuda.synchronize()
+
+    def launch(c, op, N, st):
+        L = c["L"]
+        if op == "forward":
+            L.forward(c[("X", N)], Y=c[("Y", N)], stream=st)
+        elif op == "backward_input":
+            L.backward_input(c[("dY", N)], dX=c[("dX", N)], stream=st)
+        else:
+            L.backward_weight(c[("dY", N)], c[("X", N)], dW=c[("dW", N)], stream=st)
+
+    def step(c, st):
+        for N in batches:
+            for op in OPS:
+                launch(c, op, N, st)
+
+    launches_per_step = len(batches) * len(OPS)  # every N <= 64: one kernel per op
+
+    # warm-up (also JIT-free: the library is precompiled) then capture one graph per copy
+    with torch.cuda.stream(stream):
+        for i in range(max(1, args.warmup)):
+            step(copies[i % R], stream)
+    torch.cuda.synchronize()
+    graphs = []
+    for c in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(c, stream)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    # per-op graphs: R launches of one (op, N), to time each kernel alone (L2-cold)
+    per_op = {}
+    reps = 20
+    for N in batches:
+        for op in OPS:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for c in copies:
+                    launch(c, op, N, stream)
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (reps * R)
+            b = op_bytes(op, M, K, nnz, N, s)
+            per_op[f"{op}@N={N}"] = {"us": round(us, 3), "bytes": b, "gbs": round(b / us / 1e3, 1),
+                                     "gflops": round(op_flops(nnz, N) / us / 1e3, 1)}
+            del g
+
+    # warm-up of the step graphs, then the timed region
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[i % R].replay()
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_per_step = ms / args.steps
+
+    step_bytes = sum(op_bytes(op, M, K, nnz, N, s) for N in batches for op in OPS)
+    step_flops = sum(op_flops(nnz, N) for N in batches for op in OPS)
+    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    gflops = step_flops * world / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs in, results out, every step
+    pinned = {}
+    for N in batches:
+        pinned[("X", N)] = torch.from_numpy(xs[N].view(np.int16)).view(torch.bfloat16).pin_memory()
+        pinned[("dY", N)] = torch.from_numpy(dys[N].view(np.int16)).view(torch.bfloat16).pin_memory()
+        pinned[("Y", N)] = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        pinned[("dX", N)] = torch.empty((K, N), dtype=torch.bfloat16).pin_memory()
+        pinned[("dW", N)] = torch.empty(nnz, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(pinned[("X", N)].numel() * s + pinned[("dY", N)].numel() * s for N in batches)
+    d2h = sum((pinned[("Y", N)].numel() + pinned[("dX", N)].numel() + pinned[("dW", N)].numel()) * s
+              for N in batches)
+
+    def e2e_step(c):
+        for N in batches:
+            c[("X", N)].copy_(pinned[("X", N)], non_blocking=True)
+            c[("dY", N)].copy_(pinned[("dY", N)], non_blocking=True)
+            for op in OPS:
+                launch(c, op, N, stream)
+            pinned[("Y", N)].copy_(c[("Y", N)], non_blocking=True)
+            pinned[("dX", N)].copy_(c[("dX", N)], non_blocking=True)
+            pinned[("dW", N)].copy_(c[("dW", N)], non_blocking=True)
+
+    e2e_steps = max(20, min(args.steps, 2000))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(copies[i % R])
+    torch.cuda.synchronize()
+    barrier(world)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(copies[i % R])
+        e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e_value = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+
+    # preprocessing: build (timed above, host wall clock incl. its one sync) and one restructure
+    L0 = copies[0]["L"]
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        L0.restructure(nnz // 10, seed=args.seed)
+    t_rs = time.perf_counter() - t0
+
+    pk = peaks()
+    dom_key = max(per_op, key=lambda k: per_op[k]["us"])
+    dom_op = dom_key.split("@")[0]
+    dom_launches = [k for k in per_op if k.startswith(dom_op + "@")]
+    dom_bytes = sum(per_op[k]["bytes"] for k in dom_launches)
+    dom_us = sum(per_op[k]["us"] for k in dom_launches)
+    achieved = dom_bytes / dom_us / 1e3
+    traffic = traffic_for(dom_op)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": KERNEL_NAMES[dom_op], "launches_averaged": dom_launches,
+                "peak_source": pk["source"] + " (hbm_gbs, copy burst)"}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "nnz": nnz, "batches": batches, "ops": list(OPS),
+                   "num_parts": P, "l2": f"cold: {R} rotated copies x {hot / 1e6:.1f} MB >= 3x L2 ({l2 / 2**20:.0f} MiB)",
+                   "parallelism": f"replicas x{world}"},
+        "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
+        "frac_of_nominal_8tbs": round(value / world / 8000.0, 4),
+        "gflops": round(gflops, 1),
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps},
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+        "per_op": per_op,
+        "preprocess": {"build_ms": round(t_build * 1e3, 3), "restructure_ms": round(t_rs * 1e3, 3),
+                       "restructure_drop": nnz // 10, "note": "host wall clock incl. the one status sync"},
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(layer, xs, dys, batches, budget_s=args.cpu_seconds)
+    for g in graphs:
+        del g
+    return out
+
+
+KERNEL_NAMES = {"forward": "k_spmm_small<bf16,*,*,false>", "backward_input": "k_spmm_small<bf16,*,*,true>",
+                "backward_weight": "k_sddmm_small<bf16,*,*>"}
+
+
+def traffic_for(op: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    src = os.path.join(ROOT, "sparse_spmm_b200", "csrc", "spmm.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if t.get("spmm_cu_sha256_16") != h:
+        return None
+    ent = t.get("ops", {}).get(op)
+    return ent.get("dram_bytes_per_launch_avg") if ent else None
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def _oracle_inputs(layer, xs, dys, batches):
+    import oracle
+    ref = oracle.build(layer.M, layer.K, layer.row, layer.col, layer.values, 1)
+    v64 = oracle.widen(ref["values"])
+    X64 = {N: oracle.widen(xs[N].reshape(-1)).reshape(xs[N].shape) for N in batches}
+    dY64 = {N: oracle.widen(dys[N].reshape(-1)).reshape(dys[N].shape) for N in batches}
+    return ref, v64, X64, dY64
+
+
+def _oracle_step(layer, ref, v64, X64, dY64, batches, rows_sel):
+    """One oracle step restricted to the entries of rows_sel (all three ops, every N)."""
+    import oracle
+    m = np.isin(ref["row"], rows_sel)
+    r, c, v = ref["row"][m], ref["col"][m], v64[m]
+    for N in batches:
+        oracle.forward(layer.M, layer.K, r, c, v, X64[N])
+        oracle.backward_input(layer.M, layer.K, r, c, v, dY64[N])
+        oracle.backward_weight(r, c, dY64[N], X64[N])
+    return int(m.sum())
+
+
+def cpu_baseline(layer, xs, dys, batches, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands (plain fp64 loops, 1 thread) timed on a bounded sample."""
+    ref, v64, X64, dY64 = _oracle_inputs(layer, xs, dys, batches)
+    s = 2
+    done_bytes, t_total, steps = 0, 0.0, 0
+    rng = np.random.default_rng(0)
+    frac_rows = 256
+    while t_total < budget_s and steps < 1000:
+        rows_sel = np.sort(rng.choice(layer.M, size=frac_rows, replace=False))
+        t0 = time.perf_counter()
+        n_sel = _oracle_step(layer, ref, v64, X64, dY64, batches, rows_sel)
+        t_total += time.perf_counter() - t0
+        f = frac_rows / layer.M
+        done_bytes += sum(op_bytes(op, layer.M, layer.K, layer.nnz, N, s) for N in batches for op in OPS) * \
+            (n_sel / layer.nnz) if n_sel else 0
+        steps += 1
+    return {"value": round(done_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "host_cores": len(os.sched_getaffinity(0)),
+            "sample": f"{steps} samples of {frac_rows} random rows (fwd, dX, dW at N={list(batches)}), "
+                      f"{t_total:.1f} s of oracle time; bytes scaled by the sampled share of nnz"}
+
+
+def run_reference(args, rank: int, world: int) -> dict:
+    from sparse_spmm_b200 import workloads as wl
+    layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
+    batches = [int(b) for b in args.batches.split(",")]
+    xs = {N: wl.activations(layer.K, N, "bf16", args.seed, stream=2) for N in batches}
+    dys = {N: wl.activations(layer.M, N, "bf16", args.seed, stream=3) for N in batches}
+    ref, v64, X64, dY64 = _oracle_inputs(layer, xs, dys, batches)
+    s = 2
+    full_bytes = sum(op_bytes(op, layer.M, layer.K, layer.nnz, N, s) for N in batches for op in OPS)
+    # size each step so that warm-up + steps fit in about two minutes
+    probe_rows = np.arange(0, layer.M, 64)
+    t0 = time.perf_counter()
+    n_probe = _oracle_step(layer, ref, v64, X64, dY64, batches, probe_rows)
+    t_probe = time.perf_counter() - t0
+    per_nnz = t_probe / max(n_probe, 1)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows_per_step = int(np.clip(budget / per_nnz / (layer.nnz / layer.M), 1, layer.M))
+    rng = np.random.default_rng(1)
+    for _ in range(args.warmup):
+        _oracle_step(layer, ref, v64, X64, dY64, batches, rng.choice(layer.M, rows_per_step, replace=False))
+    t_total, done = 0.0, 0.0
+    for _ in range(args.steps):
+        sel = np.sort(rng.choice(layer.M, rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        n_sel = _oracle_step(layer, ref, v64, X64, dY64, batches, sel)
+        t_total += time.perf_counter() - t0
+        done += full_bytes * n_sel / layer.nnz
+    value = done / t_total / 1e9
+    sample = f"each step: fwd, dX, dW at N={batches} over the entries of {rows_per_step} random rows of 4096"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_total / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "batches": batches, "ops": list(OPS),
+                                            "parallelism": "rank 0 only (CPU oracle)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--batches", default="1,8,32")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--parts", type=int, default=0, help="nnz-balanced parts (0 = library default)")
+    ap.add_argument("--rotate", type=int, default=0, help="number of rotated copies (0 = enough for 3x L2)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+
+    rank, world, local = dist_setup(args.gpus)
+    out = run_ours(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,672 @@
+// spmm.cu -- the three products of the truly-sparse layer on CUDA cores (sm_100a):
+//   forward      Y  = W X      (CSR walk over the row-sorted COO)
+//   transposed   dX = W^T dY   (the same kernel walking the CSC permutation)
+//   SDDMM        dW = (dY X^T) read at the stored positions
+// ("Beyond Masked Sparsity: SNACK Enables Truly Sparse Neural Networks on GPU",
+// arXiv 2610.04093, Abstract: forward and sparse backpropagation of a COO layer).
+//
+// Work split (the load-balance argument of "Two Lotteries: What It Takes to Make
+// Sparsity Fast", section on uneven work: a fixed per-unit assignment lets the busiest
+// unit set the time): the nnz are cut into P equal parts, one CTA per part, whatever
+// the row lengths.  Inside a CTA the part is cut again into equal contiguous ranges,
+// one per "worker" (G lanes that share one nnz stream and split the dense columns, NC
+// per lane).  A worker walks its range in order with a running fp32 sum per row; rows
+// that complete inside the worker are written directly.  Partial rows at worker edges
+// are combined by a segmented scan across the CTA's workers, and partial rows at CTA
+// edges by fp32 carry slots: every CTA that holds part of a split row writes its
+// partial and bumps that row's arrival counter; the last one to arrive sums the
+// partials in part order and writes the row (no waiting, deterministic order).
+// Outputs are rounded once.  No tensor cores: the gather is not a dense contraction.
+#include <algorithm>
+
+#include "internal.cuh"
+
+namespace snk {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowCap = 2048;  // row_ptr slice entries held in shared memory per CTA
+constexpr unsigned kFull = 0xffffffffu;
+
+__host__ __device__ __forceinline__ int64_t mn64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ------------------------------------------------------------------------- element I/O
+
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float load1(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load1(const __nv_bfloat16* p) {
+  return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+__device__ __forceinline__ void store1(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <int NC>
+__device__ __forceinline__ void load_vec(const float* p, float* o) {
+  if constexpr (NC == 4) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else if constexpr (NC == 2) {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+    o[0] = v.x; o[1] = v.y;
+  } else {
+    o[0] = __ldg(p);
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float* o) {
+  if constexpr (NC == 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    o[0] = lo_bf16(v.x); o[1] = hi_bf16(v.x); o[2] = lo_bf16(v.y); o[3] = hi_bf16(v.y);
+    o[4] = lo_bf16(v.z); o[5] = hi_bf16(v.z); o[6] = lo_bf16(v.w); o[7] = hi_bf16(v.w);
+  } else if constexpr (NC == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    o[0] = lo_bf16(v.x); o[1] = hi_bf16(v.x); o[2] = lo_bf16(v.y); o[3] = hi_bf16(v.y);
+  } else if constexpr (NC == 2) {
+    const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
+    o[0] = lo_bf16(v); o[1] = hi_bf16(v);
+  } else {
+    o[0] = load1(p);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int NC>
+__device__ __forceinline__ void store_vec(float* p, const float* v) {
+  if constexpr (NC == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (NC == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    p[0] = v[0];
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float* v) {
+  if constexpr (NC == 8) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  } else if constexpr (NC == 4) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  } else if constexpr (NC == 2) {
+    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v[0], v[1]);
+  } else {
+    store1(p, v[0]);
+  }
+}
+
+// lc = number of valid columns of this lane (0..NC); vec = aligned vector access allowed.
+template <int NC, typename T>
+__device__ __forceinline__ void load_cols(const T* p, int lc, bool vec, float* o) {
+  if (vec && lc == NC) {
+    load_vec<NC>(p, o);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NC; ++j) o[j] = j < lc ? load1(p + j) : 0.f;
+  }
+}
+
+template <int NC, typename T>
+__device__ __forceinline__ void store_cols(T* p, int lc, bool vec, const float* v) {
+  if (vec && lc == NC) {
+    store_vec<NC>(p, v);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NC; ++j)
+      if (j < lc) store1(p + j, v[j]);
+  }
+}
+
+// ------------------------------------------------------------------------- SpMM (fwd / transposed)
+
+template <typename T>
+struct SpmmArgs {
+  const int32_t* ptr;       // [rows + 1] row_ptr (forward) or col_ptr (transposed)
+  const int32_t* idx;       // [nnz] col (forward) or csc_row (transposed)
+  const int32_t* perm;      // [nnz] transposed only: sorted-COO index of the j-th CSC entry
+  const T* vals;            // [nnz] values in sorted-COO order
+  const int32_t* part_nnz;  // [P + 1]
+  const int32_t* part_row;  // [P + 1]
+  const T* B;               // gathered dense operand (X or dY), already offset to this launch's columns
+  T* C;                     // output (Y or dX), already offset to this launch's columns
+  int64_t ldb, ldc;
+  int64_t rows;             // output rows
+  int64_t nnz;
+  int P;
+  int ncols;                // columns in this launch (<= kCarryCols)
+  int vec;
+  float* carry_tail;        // [P][kCarryCols]
+  float* carry_head;        // [P][kCarryCols]
+  uint32_t* cnt;            // [kMaxTiles][P], zero between launches
+};
+
+template <typename T, int NC, int G, bool TRANS>
+__global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
+  constexpr int NW = kThreads / G;   // workers per CTA
+  constexpr int WPW = 32 / G;        // workers per warp
+  constexpr int NT = NC * G;         // columns per tile
+  constexpr int NWARPS = kThreads / 32;
+  constexpr int UB = NC >= 8 ? 4 : 8;  // nnz loaded ahead per worker
+  __shared__ int32_t s_rp[kRowCap];
+  __shared__ float s_agg[NWARPS][NT];
+  __shared__ int s_aggF[NWARPS];
+
+  const int part = blockIdx.x, tile = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  const int w = tid / G, l = tid % G, g = lane / G;
+  const int lane_base = lane - l;
+  const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
+
+  const int64_t a = A.part_nnz[part], b = A.part_nnz[part + 1];
+  const int64_t np = b - a;
+  const int64_t s = a + (np * w) / NW;
+  const int64_t e_end = a + (np * (w + 1)) / NW;
+
+  // values / indices of this worker's first batch, issued before the row slice arrives
+  int c[UB];
+  float v[UB];
+  auto load_batch = [&](int64_t e0, int nb) {
+#pragma unroll
+    for (int i = 0; i < UB; ++i) {
+      if (i < nb) {
+        const int64_t j = e0 + i;
+        c[i] = __ldg(A.idx + j);
+        const int64_t pe = TRANS ? (int64_t)__ldg(A.perm + j) : j;
+        v[i] = load1(A.vals + pe);
+      }
+    }
+  };
+  if (s < e_end) load_batch(s, (int)mn64(UB, e_end - s));
+
+  const int64_t ra = A.part_row[part];
+  const int64_t rb = A.part_row[part + 1];
+  const int64_t rhi = mn64(rb + 1, A.rows);
+  const int64_t span = rhi - ra + 1;
+  const bool in_smem = span <= kRowCap;
+  if (in_smem)
+    for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.ptr + ra + i);
+  __syncthreads();
+  auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.ptr + r); };
+
+  const int n0 = tile * NT + l * NC;
+  const int lc = max(0, min(NC, A.ncols - n0));
+  const bool vec = A.vec != 0;
+  const T* __restrict__ Bb = A.B + n0;
+  T* __restrict__ Cb = A.C + n0;
+  float zero[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) zero[j] = 0.f;
+
+  float acc[NC], H[NC], Tl[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) acc[j] = H[j] = Tl[j] = 0.f;
+  bool has_head = false, has_tail = false, link = true;
+  int64_t h_row = -1;
+
+  if (s < e_end) {
+    int64_t lo = ra, hi = mn64(rb, A.rows - 1);  // last r with RP(r) <= s
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (RP(mid) <= s) lo = mid; else hi = mid - 1;
+    }
+    int64_t r = lo;
+    int64_t r_end = RP(r + 1);
+    bool first = true, open = RP(r) < s;
+    if (s == 0)  // empty rows ahead of the first entry
+      for (int64_t q = 0; q < r; ++q) store_cols<NC>(Cb + q * A.ldc, lc, vec, zero);
+
+    auto finish = [&](int64_t row) {
+      if (first && open) {
+        has_head = true;
+        h_row = row;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) H[j] = acc[j];
+      } else {
+        store_cols<NC>(Cb + row * A.ldc, lc, vec, acc);
+      }
+      first = false;
+      open = false;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) acc[j] = 0.f;
+    };
+
+    int64_t e = s;
+    while (e < e_end) {
+      const int nb = (int)mn64(UB, e_end - e);
+      int cc[UB];
+      float vv[UB];
+      float x[UB][NC];
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        cc[i] = c[i];
+        vv[i] = v[i];
+      }
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        if (i < nb) load_cols<NC>(Bb + (int64_t)cc[i] * A.ldb, lc, vec, x[i]);
+      }
+      const int64_t en = e + nb;
+      if (en < e_end) load_batch(en, (int)mn64(UB, e_end - en));
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        if (i < nb) {
+          while (e + i >= r_end) {
+            finish(r);
+            ++r;
+            r_end = RP(r + 1);
+          }
+#pragma unroll
+          for (int j = 0; j < NC; ++j) acc[j] = fmaf(vv[i], x[i][j], acc[j]);
+        }
+      }
+      e = en;
+    }
+    if (r_end == e_end) {
+      finish(r);
+      link = false;
+      while (r + 1 < A.rows && RP(r + 2) == e_end) {  // empty rows right after this range
+        ++r;
+        store_cols<NC>(Cb + r * A.ldc, lc, vec, zero);
+      }
+    } else {
+      has_tail = true;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) Tl[j] = acc[j];
+      link = first && open;  // the whole range lies inside one row that started earlier
+    }
+  }
+
+  // Segmented inclusive scan of the workers' tail partials (segments = rows).
+  float S[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) S[j] = has_tail ? Tl[j] : 0.f;
+  int F = link ? 0 : 1;
+#pragma unroll
+  for (int off = 1; off < WPW; off <<= 1) {
+    float Sp[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) Sp[j] = __shfl_up_sync(kFull, S[j], off * G);
+    const int Fp = __shfl_up_sync(kFull, F, off * G);
+    if (g >= off) {
+      if (!F) {
+#pragma unroll
+        for (int j = 0; j < NC; ++j) S[j] += Sp[j];
+      }
+      F |= Fp;
+    }
+  }
+  if (g == WPW - 1) {
+#pragma unroll
+    for (int j = 0; j < NC; ++j) s_agg[wp][l * NC + j] = S[j];
+    if (l == 0) s_aggF[wp] = F;
+  }
+  __syncthreads();
+  float inc[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) inc[j] = 0.f;
+  for (int q = 0; q < wp; ++q) {
+    const int fq = s_aggF[q];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) inc[j] = fq ? s_agg[q][l * NC + j] : inc[j] + s_agg[q][l * NC + j];
+  }
+  if (!F) {
+#pragma unroll
+    for (int j = 0; j < NC; ++j) S[j] += inc[j];
+  }
+  float E[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) E[j] = __shfl_up_sync(kFull, S[j], G);
+  if (g == 0) {
+#pragma unroll
+    for (int j = 0; j < NC; ++j) E[j] = inc[j];
+  }
+
+  // Rows split across CTAs: write this CTA's partial, the last arrival combines.
+  auto cross_cta = [&](int64_t row, const float* val, bool row_ends_here) {
+    const int64_t rs = RP(row), re = RP(row + 1);
+    const int64_t P = A.P, nnz = A.nnz;
+    const int64_t p1 = ((rs + 1) * P - 1) / nnz;  // part holding the row's first entry
+    const int64_t pk = (re * P - 1) / nnz;        // part holding its last entry
+    float* slot = (row_ends_here ? A.carry_head : A.carry_tail) + (int64_t)part * kCarryCols + n0;
+#pragma unroll
+    for (int j = 0; j < NC; ++j)
+      if (j < lc) slot[j] = val[j];
+    __threadfence();
+    __syncwarp(gmask);
+    uint32_t* ctr = A.cnt + (int64_t)tile * P + p1;
+    uint32_t old = 0;
+    if (l == 0) old = atomicAdd(ctr, 1u);
+    old = __shfl_sync(gmask, old, lane_base);
+    if ((int64_t)old == pk - p1) {
+      __threadfence();
+      float sum[NC];
+#pragma unroll
+      for (int j = 0; j < NC; ++j) sum[j] = 0.f;
+      for (int64_t q = p1; q < pk; ++q) {
+        const float* src = A.carry_tail + q * kCarryCols + n0;
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+          if (j < lc) sum[j] += __ldcg(src + j);
+      }
+      const float* src = A.carry_head + pk * kCarryCols + n0;
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        if (j < lc) sum[j] += __ldcg(src + j);
+      store_cols<NC>(Cb + row * A.ldc, lc, vec, sum);
+      if (l == 0) atomicExch(ctr, 0u);
+    }
+  };
+
+  if (has_head) {
+    float val[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) val[j] = H[j] + E[j];
+    if (h_row == ra && RP(ra) < a)
+      cross_cta(h_row, val, true);
+    else
+      store_cols<NC>(Cb + h_row * A.ldc, lc, vec, val);
+  }
+  if (w == NW - 1) {
+    int64_t lo = ra, hi = mn64(rb, A.rows - 1);  // row holding entry b - 1
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (RP(mid) <= b - 1) lo = mid; else hi = mid - 1;
+    }
+    if (RP(lo + 1) > b) cross_cta(lo, S, false);
+  }
+}
+
+// ------------------------------------------------------------------------- SDDMM
+
+template <typename T>
+struct SddmmArgs {
+  const int32_t* row_ptr;
+  const int32_t* col;
+  const int32_t* part_nnz;
+  const int32_t* part_row;
+  const T* X;   // K x N
+  const T* dY;  // M x N
+  T* dW;        // [nnz]
+  int64_t ldx, lddy;
+  int64_t rows;
+  int64_t nnz;
+  int N;
+  int vec;
+};
+
+template <typename T, int NC, int G>
+__global__ void __launch_bounds__(kThreads) k_sddmm_small(const SddmmArgs<T> A) {
+  constexpr int NW = kThreads / G;
+  constexpr int NT = NC * G;
+  constexpr int UB = NC >= 8 ? 4 : 8;
+  __shared__ int32_t s_rp[kRowCap];
+
+  const int part = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int w = tid / G, l = tid % G;
+  const int lane_base = lane - l;
+  const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
+
+  const int64_t a = A.part_nnz[part], b = A.part_nnz[part + 1];
+  const int64_t np = b - a;
+  const int64_t s = a + (np * w) / NW;
+  const int64_t e_end = a + (np * (w + 1)) / NW;
+  const int64_t ra = A.part_row[part];
+  const int64_t rb = A.part_row[part + 1];
+  const int64_t rhi = mn64(rb + 1, A.rows);
+  const int64_t span = rhi - ra + 1;
+  const bool in_smem = span <= kRowCap;
+  if (in_smem)
+    for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.row_ptr + ra + i);
+  __syncthreads();
+  auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.row_ptr + r); };
+  if (s >= e_end) return;
+  const bool vec = A.vec != 0;
+
+  int64_t lo = ra, hi = mn64(rb, A.rows - 1);
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (RP(mid) <= s) lo = mid; else hi = mid - 1;
+  }
+  int64_t r = lo;
+  int64_t r_end = RP(r + 1);
+  for (int64_t e = s; e < e_end; e += UB) {
+    const int nb = (int)mn64(UB, e_end - e);
+    int cc[UB];
+    int64_t rr[UB];
+#pragma unroll
+    for (int i = 0; i < UB; ++i) {
+      cc[i] = 0;
+      rr[i] = r;
+      if (i < nb) {
+        cc[i] = __ldg(A.col + e + i);
+        while (e + i >= r_end) {
+          ++r;
+          r_end = RP(r + 1);
+        }
+        rr[i] = r;
+      }
+    }
+    float d[UB];
+#pragma unroll
+    for (int i = 0; i < UB; ++i) d[i] = 0.f;
+    for (int n0 = l * NC; n0 < A.N; n0 += NT) {
+      const int lc = min(NC, A.N - n0);
+      float xv[UB][NC], yv[UB][NC];
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        if (i < nb) {
+          load_cols<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, lc, vec, xv[i]);
+          load_cols<NC>(A.dY + rr[i] * A.lddy + n0, lc, vec, yv[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        if (i < nb) {
+#pragma unroll
+          for (int j = 0; j < NC; ++j) d[i] = fmaf(xv[i][j], yv[i][j], d[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < UB; ++i) {
+#pragma unroll
+      for (int off = G / 2; off > 0; off >>= 1) d[i] += __shfl_xor_sync(gmask, d[i], off);
+    }
+    if (l == 0) {
+#pragma unroll
+      for (int i = 0; i < UB; ++i)
+        if (i < nb) store1(A.dW + e + i, d[i]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- zero fill
+
+template <typename T>
+__global__ void k_zero_rows(T* C, int64_t rows, int64_t N, int64_t ldc) {
+  const int64_t total = rows * N;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+    store1(C + (i / N) * ldc + (i % N), 0.f);
+}
+
+// ------------------------------------------------------------------------- host dispatch
+
+int pow2ceil(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+bool aligned(const void* p, int64_t ld, int nc, int elem) {
+  return ((uintptr_t)p % (uintptr_t)(nc * elem)) == 0 && (ld % nc) == 0;
+}
+
+template <typename T, bool TRANS>
+using SpmmKernel = void (*)(const SpmmArgs<T>);
+
+template <typename T, bool TRANS>
+SpmmKernel<T, TRANS> pick_spmm(int nc, int g) {
+#define SNK_CASE(NC_, G_) \
+  if (nc == NC_ && g == G_) return k_spmm_small<T, NC_, G_, TRANS>;
+  if constexpr (sizeof(T) == 2) {
+    SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(8, 4) SNK_CASE(8, 8)
+    SNK_CASE(4, 1) SNK_CASE(2, 1)
+  } else {
+    SNK_CASE(4, 1) SNK_CASE(4, 2) SNK_CASE(4, 4) SNK_CASE(4, 8) SNK_CASE(4, 16)
+    SNK_CASE(2, 1)
+  }
+  SNK_CASE(1, 1) SNK_CASE(1, 2) SNK_CASE(1, 4) SNK_CASE(1, 8) SNK_CASE(1, 16) SNK_CASE(1, 32)
+#undef SNK_CASE
+  return nullptr;
+}
+
+template <typename T>
+using SddmmKernel = void (*)(const SddmmArgs<T>);
+
+template <typename T>
+SddmmKernel<T> pick_sddmm(int nc, int g) {
+#define SNK_CASE(NC_, G_) \
+  if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_>;
+  if constexpr (sizeof(T) == 2) {
+    SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(8, 4) SNK_CASE(8, 8) SNK_CASE(8, 16) SNK_CASE(8, 32)
+    SNK_CASE(4, 1) SNK_CASE(2, 1)
+  } else {
+    SNK_CASE(4, 1) SNK_CASE(4, 2) SNK_CASE(4, 4) SNK_CASE(4, 8) SNK_CASE(4, 16) SNK_CASE(4, 32)
+    SNK_CASE(2, 1)
+  }
+  SNK_CASE(1, 1) SNK_CASE(1, 2) SNK_CASE(1, 4) SNK_CASE(1, 8) SNK_CASE(1, 16) SNK_CASE(1, 32)
+#undef SNK_CASE
+  return nullptr;
+}
+
+template <typename T, bool TRANS>
+snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
+                      cudaStream_t s) {
+  const int elem = (int)sizeof(T);
+  const int64_t rows = TRANS ? L->K : L->M;
+  for (int64_t col0 = 0; col0 < N; col0 += kCarryCols) {
+    const int ncols = (int)std::min<int64_t>(kCarryCols, N - col0);
+    const T* Bc = B + col0;
+    T* Cc = C + col0;
+    const int ncmax = 16 / elem;
+    int nc = std::min(ncmax, pow2ceil(ncols));
+    while (nc > 1 && !(aligned(Bc, ldb, nc, elem) && aligned(Cc, ldc, nc, elem))) nc >>= 1;
+    int g = pow2ceil((ncols + nc - 1) / nc);
+    if (nc > 1) {
+      // wide vectors: the instantiated worker widths
+      const int gmax = (elem == 2) ? (nc == 8 ? 8 : 1) : (nc == 4 ? 16 : 1);
+      if (g > gmax) {
+        // fall back to narrower vectors with more lanes
+        nc = 1;
+        g = pow2ceil(ncols);
+      }
+    }
+    g = std::min(g, 32);
+    const int nt = nc * g;
+    const int tiles = (ncols + nt - 1) / nt;
+    auto kern = pick_spmm<T, TRANS>(nc, g);
+    if (kern == nullptr || tiles > kMaxTiles) return SNK_ERR_UNSUPPORTED;
+    SpmmArgs<T> A;
+    A.ptr = TRANS ? L->col_ptr : L->row_ptr;
+    A.idx = TRANS ? L->csc_row : L->col;
+    A.perm = TRANS ? L->perm : nullptr;
+    A.vals = values;
+    A.part_nnz = TRANS ? L->part_nnz_t : L->part_nnz;
+    A.part_row = TRANS ? L->part_col : L->part_row;
+    A.B = Bc;
+    A.C = Cc;
+    A.ldb = ldb;
+    A.ldc = ldc;
+    A.rows = rows;
+    A.nnz = L->nnz;
+    A.P = L->P;
+    A.ncols = ncols;
+    A.vec = nc > 1 ? 1 : 0;
+    A.carry_tail = TRANS ? L->carry_tail_b : L->carry_tail_f;
+    A.carry_head = TRANS ? L->carry_head_b : L->carry_head_f;
+    A.cnt = TRANS ? L->cnt_b : L->cnt_f;
+    kern<<<dim3((unsigned)L->P, (unsigned)tiles), kThreads, 0, s>>>(A);
+    SNK_CUDA_TRY(cudaGetLastError());
+  }
+  return SNK_OK;
+}
+
+template <typename T>
+snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* X, int64_t ldx, int64_t N, T* dW,
+                       cudaStream_t s) {
+  const int elem = (int)sizeof(T);
+  const int ncmax = 16 / elem;
+  int nc = std::min<int64_t>(ncmax, pow2ceil((int)std::min<int64_t>(N, 1 << 20)));
+  while (nc > 1 && !(aligned(X, ldx, nc, elem) && aligned(dY, lddy, nc, elem))) nc >>= 1;
+  int g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>((N + nc - 1) / nc, 64)));
+  auto kern = pick_sddmm<T>(nc, g);
+  if (kern == nullptr) {
+    nc = 1;
+    g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>(N, 64)));
+    kern = pick_sddmm<T>(nc, g);
+  }
+  if (kern == nullptr) return SNK_ERR_UNSUPPORTED;
+  SddmmArgs<T> A;
+  A.row_ptr = L->row_ptr;
+  A.col = L->col;
+  A.part_nnz = L->part_nnz;
+  A.part_row = L->part_row;
+  A.X = X;
+  A.dY = dY;
+  A.dW = dW;
+  A.ldx = ldx;
+  A.lddy = lddy;
+  A.rows = L->M;
+  A.nnz = L->nnz;
+  A.N = (int)N;
+  A.vec = nc > 1 ? 1 : 0;
+  kern<<<(unsigned)L->P, kThreads, 0, s>>>(A);
+  SNK_CUDA_TRY(cudaGetLastError());
+  return SNK_OK;
+}
+
+}  // namespace
+
+snk_status launch_zero_rows(void* C, int64_t rows, int64_t N, int64_t ldc, int elem_bytes, cudaStream_t s) {
+  if (rows <= 0 || N <= 0) return SNK_OK;
+  const int64_t total = rows * N;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, 65535 * 4);
+  if (elem_bytes == 4)
+    k_zero_rows<float><<<grid, 256, 0, s>>>((float*)C, rows, N, ldc);
+  else
+    k_zero_rows<__nv_bfloat16><<<grid, 256, 0, s>>>((__nv_bfloat16*)C, rows, N, ldc);
+  SNK_CUDA_TRY(cudaGetLastError());
+  return SNK_OK;
+}
+
+snk_status launch_spmm(const snk_layout* L, bool transpose, const void* values, const void* B, int64_t N, int64_t ldb,
+                       void* C, int64_t ldc, cudaStream_t s) {
+  const int64_t rows = transpose ? L->K : L->M;
+  if (L->nnz == 0) return launch_zero_rows(C, rows, N, ldc, L->dtype == SNK_F32 ? 4 : 2, s);
+  if (L->dtype == SNK_F32) {
+    return transpose ? spmm_typed<float, true>(L, (const float*)values, (const float*)B, N, ldb, (float*)C, ldc, s)
+                     : spmm_typed<float, false>(L, (const float*)values, (const float*)B, N, ldb, (float*)C, ldc, s);
+  }
+  using bf = __nv_bfloat16;
+  return transpose ? spmm_typed<bf, true>(L, (const bf*)values, (const bf*)B, N, ldb, (bf*)C, ldc, s)
+                   : spmm_typed<bf, false>(L, (const bf*)values, (const bf*)B, N, ldb, (bf*)C, ldc, s);
+}
+
+snk_status launch_sddmm(const snk_layout* L, const void* dY, int64_t lddy, const void* X, int64_t ldx, int64_t N,
+                        void* dW, cudaStream_t s) {
+  if (L->nnz == 0) return SNK_OK;
+  if (L->dtype == SNK_F32)
+    return sddmm_typed<float>(L, (const float*)dY, lddy, (const float*)X, ldx, N, (float*)dW, s);
+  using bf = __nv_bfloat16;
+  return sddmm_typed<bf>(L, (const bf*)dY, lddy, (const bf*)X, ldx, N, (bf*)dW, s);
+}
+
+}  // namespace snk

@@ -1,0 +1,279 @@
+"""Thin ctypes binding of libsnk.so (the C ABI declared in include/snk.h).
+
+Argument marshalling only: torch tensors supply device memory and the current CUDA stream,
+and every step of the layer runs in the library's kernels.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+
+Low-level functions carry the C names (``snk_build``, ``snk_forward``, ...).  ``Layout``
+bundles a built layout with its workspace tensor for convenience.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsnk.so")
+
+SNK_F32, SNK_BF16 = 0, 1
+_STATUS = ["SNK_OK", "SNK_ERR_INVALID_ARG", "SNK_ERR_OUT_OF_RANGE", "SNK_ERR_DUPLICATE",
+           "SNK_ERR_WORKSPACE_TOO_SMALL", "SNK_ERR_UNSUPPORTED", "SNK_ERR_INVALID_VALUE",
+           "SNK_ERR_NO_ROOM", "SNK_ERR_TIMEOUT", "SNK_ERR_CUDA"]
+
+EXPORTED = ("snk_status_string", "snk_default_num_parts", "snk_workspace_bytes", "snk_build",
+            "snk_forward", "snk_backward_input", "snk_backward_weight", "snk_restructure",
+            "snk_layout_info", "snk_destroy")
+
+
+class SnkError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        name = _STATUS[code] if 0 <= code < len(_STATUS) else str(code)
+        super().__init__(f"{where}: {name}" if where else name)
+        self.code = code
+        self.status = name
+
+
+class _View(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("nnz", ctypes.c_int64),
+                ("num_parts", ctypes.c_int32), ("dtype", ctypes.c_int32), ("device", ctypes.c_int32)] + \
+               [(n, ctypes.c_void_p) for n in ("row", "col", "row_ptr", "col_ptr", "csc_row", "perm",
+                                               "part_nnz", "part_row", "part_nnz_t", "part_col")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libsnk.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m sparse_spmm_b200.build`")
+    lib = ctypes.CDLL(path)
+    i64, i32, vp, u64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_uint64
+    st = ctypes.c_int
+    lib.snk_status_string.restype = ctypes.c_char_p
+    lib.snk_status_string.argtypes = [st]
+    lib.snk_default_num_parts.restype = i32
+    lib.snk_default_num_parts.argtypes = [i64, i32]
+    lib.snk_workspace_bytes.restype = ctypes.c_size_t
+    lib.snk_workspace_bytes.argtypes = [i64, i64, i64, i32]
+    lib.snk_build.restype = st
+    lib.snk_build.argtypes = [i64, i64, i64, vp, vp, vp, st, i32, vp, ctypes.c_size_t, vp,
+                              ctypes.POINTER(vp)]
+    lib.snk_forward.restype = st
+    lib.snk_forward.argtypes = [vp, vp, vp, i64, i64, vp, i64, st, vp]
+    lib.snk_backward_input.restype = st
+    lib.snk_backward_input.argtypes = [vp, vp, vp, i64, i64, vp, i64, st, vp]
+    lib.snk_backward_weight.restype = st
+    lib.snk_backward_weight.argtypes = [vp, vp, i64, vp, i64, i64, vp, st, vp]
+    lib.snk_restructure.restype = st
+    lib.snk_restructure.argtypes = [vp, vp, i64, u64, ctypes.c_float, vp, vp]
+    lib.snk_layout_info.restype = st
+    lib.snk_layout_info.argtypes = [vp, ctypes.POINTER(_View)]
+    lib.snk_destroy.restype = None
+    lib.snk_destroy.argtypes = [vp]
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return SNK_F32
+    if t == torch.bfloat16:
+        return SNK_BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise SnkError(code, where)
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("dense operands must be 2-D with unit column stride")
+    return t.stride(0)
+
+
+# ----------------------------------------------------------------------------- C-named calls
+
+def snk_status_string(code: int) -> str:
+    return load_library().snk_status_string(code).decode()
+
+
+def snk_default_num_parts(nnz: int, sm_count: int) -> int:
+    return int(load_library().snk_default_num_parts(nnz, sm_count))
+
+
+def snk_workspace_bytes(M: int, K: int, nnz: int, num_parts: int = 0) -> int:
+    return int(load_library().snk_workspace_bytes(M, K, nnz, num_parts))
+
+
+def snk_build(M, K, row, col, values, num_parts, workspace, stream=None):
+    """Sorts row/col/values in place and returns an opaque layout handle (c_void_p)."""
+    out = ctypes.c_void_p()
+    nnz = row.numel()
+    code = load_library().snk_build(M, K, nnz, _ptr(row), _ptr(col), _ptr(values), _dtype_code(values.dtype),
+                                    num_parts, _ptr(workspace), workspace.numel(), _stream(stream),
+                                    ctypes.byref(out))
+    _check(code, "snk_build")
+    return out
+
+
+def snk_forward(handle, values, X, N, ldx, Y, ldy, stream=None):
+    _check(load_library().snk_forward(handle, _ptr(values), _ptr(X), N, ldx, _ptr(Y), ldy,
+                                      _dtype_code(X.dtype), _stream(stream)), "snk_forward")
+
+
+def snk_backward_input(handle, values, dY, N, lddy, dX, lddx, stream=None):
+    _check(load_library().snk_backward_input(handle, _ptr(values), _ptr(dY), N, lddy, _ptr(dX), lddx,
+                                             _dtype_code(dY.dtype), _stream(stream)), "snk_backward_input")
+
+
+def snk_backward_weight(handle, dY, lddy, X, ldx, N, dW, stream=None):
+    _check(load_library().snk_backward_weight(handle, _ptr(dY), lddy, _ptr(X), ldx, N, _ptr(dW),
+                                              _dtype_code(X.dtype), _stream(stream)), "snk_backward_weight")
+
+
+def snk_restructure(handle, values, drop_count, seed, regrow_value=0.0, old_to_new=None, stream=None):
+    _check(load_library().snk_restructure(handle, _ptr(values), drop_count, seed, regrow_value,
+                                          _ptr(old_to_new), _stream(stream)), "snk_restructure")
+
+
+def snk_layout_info(handle) -> _View:
+    v = _View()
+    _check(load_library().snk_layout_info(handle, ctypes.byref(v)), "snk_layout_info")
+    return v
+
+
+def snk_destroy(handle):
+    if handle:
+        load_library().snk_destroy(handle)
+
+
+# ----------------------------------------------------------------------------- convenience
+
+class Layout:
+    """A built layout plus the workspace tensor that backs it.
+
+    ``row``, ``col`` (int32) and ``values`` (float32 or bfloat16) are CUDA tensors; they are
+    sorted in place by the build and must stay alive with the layout.
+    """
+
+    def __init__(self, M: int, K: int, row: torch.Tensor, col: torch.Tensor, values: torch.Tensor,
+                 num_parts: int = 0, stream=None):
+        if row.dtype != torch.int32 or col.dtype != torch.int32:
+            raise TypeError("row/col must be int32")
+        if not (row.is_cuda and col.is_cuda and values.is_cuda):
+            raise ValueError("row, col and values must be CUDA tensors")
+        if not (row.is_contiguous() and col.is_contiguous() and values.is_contiguous()):
+            raise ValueError("row, col and values must be contiguous")
+        self.M, self.K = int(M), int(K)
+        self.row, self.col, self.values = row, col, values
+        self.dtype = values.dtype
+        nbytes = snk_workspace_bytes(self.M, self.K, row.numel(), num_parts)
+        if nbytes == 0:
+            raise SnkError(1, "snk_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=row.device)
+        self.handle = snk_build(self.M, self.K, row, col, values, num_parts, self.workspace, stream)
+        info = snk_layout_info(self.handle)
+        self.nnz = int(info.nnz)
+        self.num_parts = int(info.num_parts)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            snk_destroy(h)
+            self.handle = None
+
+    def close(self):
+        self.__del__()
+
+    # -- products
+    def forward(self, X: torch.Tensor, Y: torch.Tensor | None = None, values=None, stream=None):
+        values = self.values if values is None else values
+        N = X.shape[1]
+        if Y is None:
+            Y = torch.empty((self.M, N), dtype=X.dtype, device=X.device)
+        snk_forward(self.handle, values, X, N, _ld(X), Y, _ld(Y), stream)
+        return Y
+
+    def backward_input(self, dY: torch.Tensor, dX: torch.Tensor | None = None, values=None, stream=None):
+        values = self.values if values is None else values
+        N = dY.shape[1]
+        if dX is None:
+            dX = torch.empty((self.K, N), dtype=dY.dtype, device=dY.device)
+        snk_backward_input(self.handle, values, dY, N, _ld(dY), dX, _ld(dX), stream)
+        return dX
+
+    def backward_weight(self, dY: torch.Tensor, X: torch.Tensor, dW: torch.Tensor | None = None, stream=None):
+        N = X.shape[1]
+        if dW is None:
+            dW = torch.empty(self.nnz, dtype=X.dtype, device=X.device)
+        snk_backward_weight(self.handle, dY, _ld(dY), X, _ld(X), N, dW, stream)
+        return dW
+
+    def restructure(self, drop_count: int, seed: int, regrow_value: float = 0.0, want_map: bool = True,
+                    stream=None):
+        o2n = torch.empty(self.nnz, dtype=torch.int32, device=self.row.device) if want_map else None
+        snk_restructure(self.handle, self.values, drop_count, seed, regrow_value, o2n, stream)
+        return o2n
+
+    # -- inspection
+    def arrays(self) -> dict:
+        """Device arrays of the layout as int32 tensors (views of the workspace)."""
+        v = snk_layout_info(self.handle)
+        base = self.workspace.data_ptr()
+        ws32 = self.workspace.view(torch.int32) if self.workspace.numel() % 4 == 0 else None
+
+        def sl(ptr, n):
+            off = ptr - base
+            assert off % 4 == 0 and ws32 is not None
+            return ws32[off // 4: off // 4 + n]
+
+        P = int(v.num_parts)
+        return {
+            "row": self.row, "col": self.col, "values": self.values,
+            "row_ptr": sl(v.row_ptr, self.M + 1), "col_ptr": sl(v.col_ptr, self.K + 1),
+            "csc_row": sl(v.csc_row, self.nnz), "perm": sl(v.perm, self.nnz),
+            "part_nnz": sl(v.part_nnz, P + 1), "part_row": sl(v.part_row, P + 1),
+            "part_nnz_t": sl(v.part_nnz_t, P + 1), "part_col": sl(v.part_col, P + 1),
+            "num_parts": P,
+        }
+
+
+class SparseLinearFunction(torch.autograd.Function):
+    """Y = W X with W held by a Layout; backward returns dX = W^T dY and dW (per entry).
+
+    Inputs: values (the layout's value tensor, the trainable parameter), X (K x N).
+    """
+
+    @staticmethod
+    def forward(ctx, values, X, layout):
+        ctx.layout = layout
+        ctx.save_for_backward(values, X)
+        return layout.forward(X.contiguous(), values=values)
+
+    @staticmethod
+    def backward(ctx, dY):
+        values, X = ctx.saved_tensors
+        L = ctx.layout
+        dY = dY.contiguous()
+        dX = L.backward_input(dY, values=values) if ctx.needs_input_grad[1] else None
+        dW = L.backward_weight(dY, X) if ctx.needs_input_grad[0] else None
+        return dW, dX, None
