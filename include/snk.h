@@ -84,7 +84,8 @@ typedef struct {
 SNK_API const char* snk_status_string(snk_status s);
 
 /* Default number of nnz-balanced parts for `nnz` entries on a GPU with `sm_count` SMs:
- * min(4 * sm_count, ceil(nnz / 256)), at least 1.  Pure host arithmetic. */
+ * min(3 * sm_count, ceil(nnz / 256)), at least 1 (the product kernels keep three CTAs of
+ * 256 threads resident per SM, so the default is one wave).  Pure host arithmetic. */
 SNK_API int32_t snk_default_num_parts(int64_t nnz, int32_t sm_count);
 
 /* Bytes of device workspace a layout with these sizes needs (num_parts as passed to

@@ -298,6 +298,42 @@ __global__ void k_parts(const int32_t* __restrict__ ptr, int64_t dim, int64_t nn
   }
 }
 
+// Last r in [lo, dim] with ptr[r] <= x (the row holding entry x when x < nnz).
+__device__ __forceinline__ int64_t row_holding(const int32_t* __restrict__ ptr, int64_t lo, int64_t dim, int64_t x) {
+  int64_t hi = dim;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (ptr[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Work descriptor of part p for the product kernels.  The part's nominal range
+// [a, b) = [floor(p nnz / P), floor((p+1) nnz / P)) is moved to row boundaries where a
+// row shorter than the smallest part crosses it: such a row belongs wholly to the part in
+// which it starts (that part extends its end, the next one skips the row's remainder),
+// so only rows longer than a part are ever split between CTAs.  desc = {a', b', ra, rb}
+// with ra the row holding a' and rb the row holding b' (dim when b' == nnz).
+__global__ void k_part_desc(const int32_t* __restrict__ ptr, int64_t dim, int64_t nnz, int P,
+                            const int32_t* __restrict__ part_idx, int4* __restrict__ desc, const uint32_t* err) {
+  if (*err) return;
+  for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < P; p += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t a = (p * nnz) / P, b = ((p + 1) * nnz) / P;
+    const int64_t lmax = nnz / P;
+    int64_t a2 = a, b2 = b;
+    if (a < b) {
+      const int64_t ra = part_idx[p];
+      if (ptr[ra] < a && ptr[ra + 1] - ptr[ra] <= lmax) a2 = ptr[ra + 1];
+      const int64_t t = row_holding(ptr, ra, dim - 1, b - 1);
+      if (ptr[t + 1] > b && ptr[t + 1] - ptr[t] <= lmax) b2 = ptr[t + 1];
+      if (a2 > b2) a2 = b2;
+    }
+    const int64_t ra2 = a2 < nnz ? row_holding(ptr, 0, dim - 1, a2) : dim;
+    const int64_t rb2 = b2 < nnz ? row_holding(ptr, 0, dim - 1, b2) : dim;
+    desc[p] = make_int4((int)a2, (int)b2, (int)ra2, (int)rb2);
+  }
+}
+
 // ------------------------------------------------------------------------- restructure kernels
 
 template <typename W>
@@ -507,6 +543,8 @@ size_t carve(snk_layout* L, uint8_t* base) {
   L->part_row = c.take<int32_t>(P + 1);
   L->part_nnz_t = c.take<int32_t>(P + 1);
   L->part_col = c.take<int32_t>(P + 1);
+  L->desc_f = c.take<int4>(P);
+  L->desc_t = c.take<int4>(P);
   L->carry_tail_f = c.take<float>(P * kCarryCols);
   L->carry_head_f = c.take<float>(P * kCarryCols);
   L->cnt_f = c.take<uint32_t>((int64_t)kMaxTiles * P);
@@ -562,6 +600,8 @@ snk_status derive_format(snk_layout* L, cudaStream_t s) {
                                                             L->err);
   k_parts<<<grid_for(L->P + 1, kThreads), kThreads, 0, s>>>(L->col_ptr, L->K, nnz, L->P, L->part_nnz_t, L->part_col,
                                                             L->err);
+  k_part_desc<<<grid_for(L->P, kThreads), kThreads, 0, s>>>(L->row_ptr, L->M, nnz, L->P, L->part_row, L->desc_f, L->err);
+  k_part_desc<<<grid_for(L->P, kThreads), kThreads, 0, s>>>(L->col_ptr, L->K, nnz, L->P, L->part_col, L->desc_t, L->err);
   SNK_CUDA_TRY(cudaGetLastError());
   SNK_CUDA_TRY(fill_u32(L->cnt_f, (int64_t)kMaxTiles * L->P, 0u, s));
   SNK_CUDA_TRY(fill_u32(L->cnt_b, (int64_t)kMaxTiles * L->P, 0u, s));

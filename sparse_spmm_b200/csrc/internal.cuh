@@ -52,6 +52,10 @@ struct snk_layout {
   int32_t* part_row;
   int32_t* part_nnz_t;
   int32_t* part_col;
+  // per-CTA work descriptors of the products, one int4 per part: {a, b, ra, rb} = the
+  // entry range the CTA walks and the rows holding a and b (see k_part_desc).
+  int4* desc_f;
+  int4* desc_t;
   // cross-CTA carries of the forward / transposed kernels: [P][kCarryCols] tail and head
   // slots, and [kMaxTiles][P] arrival counters (zero between launches).
   float* carry_tail_f;

@@ -51,7 +51,7 @@ const char* snk_status_string(snk_status s) {
 int32_t snk_default_num_parts(int64_t nnz, int32_t sm_count) {
   if (sm_count < 1) sm_count = 1;
   const int64_t by_size = (nnz + 255) / 256;
-  int64_t p = std::min<int64_t>(4 * (int64_t)sm_count, by_size);
+  int64_t p = std::min<int64_t>(3 * (int64_t)sm_count, by_size);
   return (int32_t)std::max<int64_t>(p, 1);
 }
 

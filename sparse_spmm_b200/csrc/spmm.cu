@@ -8,15 +8,20 @@
 // Work split (the load-balance argument of "Two Lotteries: What It Takes to Make
 // Sparsity Fast", section on uneven work: a fixed per-unit assignment lets the busiest
 // unit set the time): the nnz are cut into P equal parts, one CTA per part, whatever
-// the row lengths.  Inside a CTA the part is cut again into equal contiguous ranges,
-// one per "worker" (G lanes that share one nnz stream and split the dense columns, NC
-// per lane).  A worker walks its range in order with a running fp32 sum per row; rows
-// that complete inside the worker are written directly.  Partial rows at worker edges
-// are combined by a segmented scan across the CTA's workers, and partial rows at CTA
-// edges by fp32 carry slots: every CTA that holds part of a split row writes its
-// partial and bumps that row's arrival counter; the last one to arrive sums the
-// partials in part order and writes the row (no waiting, deterministic order).
-// Outputs are rounded once.  No tensor cores: the gather is not a dense contraction.
+// the row lengths; a precomputed descriptor moves each part's ends to row boundaries
+// unless the row there is longer than a part.  Inside a CTA the range is cut again into
+// equal contiguous pieces, one per "worker" (G lanes that share one entry stream and
+// split the dense columns, NC per lane).  A worker walks its piece in order with a
+// running fp32 sum per row; rows that complete inside the worker are written directly.
+// Partial rows at worker edges are combined by a segmented scan across the CTA's
+// workers, and partial rows at CTA edges (long rows only) by fp32 carry slots: every CTA
+// holding part of such a row writes its partial and bumps that row's arrival counter;
+// the last one to arrive sums the partials in part order and writes the row (no waiting,
+// deterministic order).  Outputs are rounded once.  No tensor cores: the gather is not a
+// dense contraction.
+//
+// Gathered rows of the dense operand are kept packed (bf16 pairs in 32-bit words) until
+// the FMA and are multiplied with packed fp32 FMAs (two lanes of fp32 per instruction).
 #include <algorithm>
 
 #include "internal.cuh"
@@ -25,15 +30,16 @@ namespace snk {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRowCap = 2048;  // row_ptr slice entries held in shared memory per CTA
+constexpr int kRowCap = 2048;   // row_ptr slice entries held in shared memory per CTA
+constexpr int kStageCap = 4096; // SDDMM results staged in shared memory per CTA
 constexpr unsigned kFull = 0xffffffffu;
 
 __host__ __device__ __forceinline__ int64_t mn64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 // ------------------------------------------------------------------------- element I/O
 
-__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 __device__ __forceinline__ float load1(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float load1(const __nv_bfloat16* p) {
@@ -42,33 +48,72 @@ __device__ __forceinline__ float load1(const __nv_bfloat16* p) {
 __device__ __forceinline__ void store1(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-template <int NC>
-__device__ __forceinline__ void load_vec(const float* p, float* o) {
-  if constexpr (NC == 4) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-  } else if constexpr (NC == 2) {
-    const float2 v = __ldg(reinterpret_cast<const float2*>(p));
-    o[0] = v.x; o[1] = v.y;
+// NC consecutive elements of T held as loaded: 32-bit words (two bf16 per word, or one
+// float).  NC > 1 loads are single aligned vector loads (the host guarantees alignment).
+template <typename T, int NC>
+struct Packed {
+  static constexpr int W = sizeof(T) == 2 ? (NC + 1) / 2 : NC;
+  uint32_t w[W];
+};
+
+template <int NC, typename T>
+__device__ __forceinline__ void load_packed(const T* p, Packed<T, NC>& r) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (NC == 8) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+      r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+    } else if constexpr (NC == 4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      r.w[0] = v.x; r.w[1] = v.y;
+    } else if constexpr (NC == 2) {
+      r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+    } else {
+      r.w[0] = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16;  // one value, high half
+    }
   } else {
-    o[0] = __ldg(p);
+    if constexpr (NC == 4) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+      r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+    } else if constexpr (NC == 2) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      r.w[0] = v.x; r.w[1] = v.y;
+    } else {
+      r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+    }
   }
 }
 
-template <int NC>
-__device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float* o) {
-  if constexpr (NC == 8) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-    o[0] = lo_bf16(v.x); o[1] = hi_bf16(v.x); o[2] = lo_bf16(v.y); o[3] = hi_bf16(v.y);
-    o[4] = lo_bf16(v.z); o[5] = hi_bf16(v.z); o[6] = lo_bf16(v.w); o[7] = hi_bf16(v.w);
-  } else if constexpr (NC == 4) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-    o[0] = lo_bf16(v.x); o[1] = hi_bf16(v.x); o[2] = lo_bf16(v.y); o[3] = hi_bf16(v.y);
-  } else if constexpr (NC == 2) {
-    const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
-    o[0] = lo_bf16(v); o[1] = hi_bf16(v);
+template <typename T, int NC>
+__device__ __forceinline__ void zero_packed(Packed<T, NC>& r) {
+#pragma unroll
+  for (int k = 0; k < Packed<T, NC>::W; ++k) r.w[k] = 0u;
+}
+
+// Unpacked value j of a packed group.
+template <typename T, int NC>
+__device__ __forceinline__ float unpack(const Packed<T, NC>& r, int j) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (NC == 1) return __uint_as_float(r.w[0]);
+    return (j & 1) ? bf_hi(r.w[j >> 1]) : bf_lo(r.w[j >> 1]);
   } else {
-    o[0] = load1(p);
+    return __uint_as_float(r.w[j]);
+  }
+}
+
+// acc[j] += v * x[j] for the NC columns, two columns per packed fp32 FMA.
+template <typename T, int NC>
+__device__ __forceinline__ void fma_row(float v, const Packed<T, NC>& x, float* acc) {
+  if constexpr (NC == 1) {
+    acc[0] = fmaf(v, unpack<T, NC>(x, 0), acc[0]);
+  } else {
+    const float2 vv = make_float2(v, v);
+#pragma unroll
+    for (int j = 0; j < NC; j += 2) {
+      float2 a2 = make_float2(acc[j], acc[j + 1]);
+      a2 = __ffma2_rn(vv, make_float2(unpack<T, NC>(x, j), unpack<T, NC>(x, j + 1)), a2);
+      acc[j] = a2.x;
+      acc[j + 1] = a2.y;
+    }
   }
 }
 
@@ -77,99 +122,112 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int NC>
-__device__ __forceinline__ void store_vec(float* p, const float* v) {
-  if constexpr (NC == 4) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  } else if constexpr (NC == 2) {
-    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
-  } else {
-    p[0] = v[0];
-  }
-}
-
-template <int NC>
-__device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float* v) {
-  if constexpr (NC == 8) {
-    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-  } else if constexpr (NC == 4) {
-    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
-  } else if constexpr (NC == 2) {
-    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v[0], v[1]);
-  } else {
-    store1(p, v[0]);
-  }
-}
-
-// lc = number of valid columns of this lane (0..NC); vec = aligned vector access allowed.
+// Store NC values (rounded once to T).  NC > 1 stores are single aligned vector stores.
 template <int NC, typename T>
-__device__ __forceinline__ void load_cols(const T* p, int lc, bool vec, float* o) {
-  if (vec && lc == NC) {
-    load_vec<NC>(p, o);
+__device__ __forceinline__ void store_cols(T* p, const float* v) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (NC == 8) {
+      *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    } else if constexpr (NC == 4) {
+      *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    } else if constexpr (NC == 2) {
+      *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v[0], v[1]);
+    } else {
+      store1(p, v[0]);
+    }
   } else {
-#pragma unroll
-    for (int j = 0; j < NC; ++j) o[j] = j < lc ? load1(p + j) : 0.f;
+    if constexpr (NC == 4) {
+      *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (NC == 2) {
+      *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    } else {
+      p[0] = v[0];
+    }
   }
 }
 
 template <int NC, typename T>
-__device__ __forceinline__ void store_cols(T* p, int lc, bool vec, const float* v) {
-  if (vec && lc == NC) {
-    store_vec<NC>(p, v);
-  } else {
+__device__ __forceinline__ void store_zero(T* p) {
+  float z[NC];
 #pragma unroll
-    for (int j = 0; j < NC; ++j)
-      if (j < lc) store1(p + j, v[j]);
+  for (int j = 0; j < NC; ++j) z[j] = 0.f;
+  store_cols<NC>(p, z);
+}
+
+// ------------------------------------------------------------------------- launch ordering
+
+// Programmatic dependent launch: every product kernel lets the next kernel in the stream
+// start launching at once, and waits for the previous grid (and its memory) before it
+// touches global memory, since any input may have been written by that grid.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Last r in [lo, hi] with rp(r) <= x.
+template <typename RPF>
+__device__ __forceinline__ int64_t search_row(RPF rp, int64_t lo, int64_t hi, int64_t x) {
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (rp(mid) <= x) lo = mid; else hi = mid - 1;
   }
+  return lo;
 }
 
 // ------------------------------------------------------------------------- SpMM (fwd / transposed)
 
 template <typename T>
 struct SpmmArgs {
-  const int32_t* ptr;       // [rows + 1] row_ptr (forward) or col_ptr (transposed)
-  const int32_t* idx;       // [nnz] col (forward) or csc_row (transposed)
-  const int32_t* perm;      // [nnz] transposed only: sorted-COO index of the j-th CSC entry
-  const T* vals;            // [nnz] values in sorted-COO order
-  const int32_t* part_nnz;  // [P + 1]
-  const int32_t* part_row;  // [P + 1]
-  const T* B;               // gathered dense operand (X or dY), already offset to this launch's columns
-  T* C;                     // output (Y or dX), already offset to this launch's columns
+  const int32_t* ptr;  // [rows + 1] row_ptr (forward) or col_ptr (transposed)
+  const int32_t* idx;  // [nnz] col (forward) or csc_row (transposed)
+  const int32_t* perm; // [nnz] transposed only: sorted-COO index of the j-th CSC entry
+  const T* vals;       // [nnz] values in sorted-COO order
+  const int4* desc;    // [P] per-CTA work descriptors {a, b, ra, rb}
+  const T* B;          // gathered dense operand (X or dY), offset to this launch's columns
+  T* C;                // output (Y or dX), offset to this launch's columns
   int64_t ldb, ldc;
-  int64_t rows;             // output rows
+  int64_t rows;        // output rows
   int64_t nnz;
   int P;
-  int ncols;                // columns in this launch (<= kCarryCols)
-  int vec;
-  float* carry_tail;        // [P][kCarryCols]
-  float* carry_head;        // [P][kCarryCols]
-  uint32_t* cnt;            // [kMaxTiles][P], zero between launches
+  int ncols;           // columns in this launch (<= kCarryCols, a multiple of NC)
+  float* carry_tail;   // [P][kCarryCols]
+  float* carry_head;   // [P][kCarryCols]
+  uint32_t* cnt;       // [kMaxTiles][P], zero between launches
 };
 
+// Entries in flight per worker: as many as the register budget of 3 CTAs per SM allows.
+template <typename T, int NC>
+constexpr int spmm_batch() { return NC * (int)sizeof(T) >= 16 ? 4 : 8; }
+template <typename T, int NC>
+constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 8 ? 4 : 6; }
+
 template <typename T, int NC, int G, bool TRANS>
-__global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
+__global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A) {
   constexpr int NW = kThreads / G;   // workers per CTA
   constexpr int WPW = 32 / G;        // workers per warp
   constexpr int NT = NC * G;         // columns per tile
   constexpr int NWARPS = kThreads / 32;
-  constexpr int UB = NC >= 8 ? 4 : 8;  // nnz loaded ahead per worker
+  constexpr int UB = spmm_batch<T, NC>();
   __shared__ int32_t s_rp[kRowCap];
   __shared__ float s_agg[NWARPS][NT];
   __shared__ int s_aggF[NWARPS];
 
+  pdl_launch_dependents();
   const int part = blockIdx.x, tile = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   const int w = tid / G, l = tid % G, g = lane / G;
   const int lane_base = lane - l;
   const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
+  const int n0 = tile * NT + l * NC;
+  const bool active = n0 < A.ncols;  // this lane holds NC real columns (or none)
+  pdl_wait();
 
-  const int64_t a = A.part_nnz[part], b = A.part_nnz[part + 1];
+  const int4 dsc = __ldg(A.desc + part);
+  const int64_t a = dsc.x, b = dsc.y, ra = dsc.z, rb = dsc.w;
   const int64_t np = b - a;
   const int64_t s = a + (np * w) / NW;
   const int64_t e_end = a + (np * (w + 1)) / NW;
 
-  // values / indices of this worker's first batch, issued before the row slice arrives
+  // the worker's next batch of indices / values (prefetched one batch ahead)
   int c[UB];
   float v[UB];
   auto load_batch = [&](int64_t e0, int nb) {
@@ -185,42 +243,29 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
   };
   if (s < e_end) load_batch(s, (int)mn64(UB, e_end - s));
 
-  const int64_t ra = A.part_row[part];
-  const int64_t rb = A.part_row[part + 1];
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
-  const bool in_smem = span <= kRowCap;
+  const bool in_smem = np > 0 && span <= kRowCap;
   if (in_smem)
     for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.ptr + ra + i);
   __syncthreads();
   auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.ptr + r); };
 
-  const int n0 = tile * NT + l * NC;
-  const int lc = max(0, min(NC, A.ncols - n0));
-  const bool vec = A.vec != 0;
   const T* __restrict__ Bb = A.B + n0;
   T* __restrict__ Cb = A.C + n0;
-  float zero[NC];
-#pragma unroll
-  for (int j = 0; j < NC; ++j) zero[j] = 0.f;
 
-  float acc[NC], H[NC], Tl[NC];
+  float acc[NC], H[NC];
 #pragma unroll
-  for (int j = 0; j < NC; ++j) acc[j] = H[j] = Tl[j] = 0.f;
+  for (int j = 0; j < NC; ++j) acc[j] = H[j] = 0.f;
   bool has_head = false, has_tail = false, link = true;
   int64_t h_row = -1;
 
   if (s < e_end) {
-    int64_t lo = ra, hi = mn64(rb, A.rows - 1);  // last r with RP(r) <= s
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (RP(mid) <= s) lo = mid; else hi = mid - 1;
-    }
-    int64_t r = lo;
+    int64_t r = search_row(RP, ra, mn64(rb, A.rows - 1), s);
     int64_t r_end = RP(r + 1);
     bool first = true, open = RP(r) < s;
-    if (s == 0)  // empty rows ahead of the first entry
-      for (int64_t q = 0; q < r; ++q) store_cols<NC>(Cb + q * A.ldc, lc, vec, zero);
+    if (s == 0 && active)  // empty rows ahead of the first entry
+      for (int64_t q = 0; q < r; ++q) store_zero<NC>(Cb + q * A.ldc);
 
     auto finish = [&](int64_t row) {
       if (first && open) {
@@ -228,8 +273,8 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
         h_row = row;
 #pragma unroll
         for (int j = 0; j < NC; ++j) H[j] = acc[j];
-      } else {
-        store_cols<NC>(Cb + row * A.ldc, lc, vec, acc);
+      } else if (active) {
+        store_cols<NC>(Cb + row * A.ldc, acc);
       }
       first = false;
       open = false;
@@ -240,30 +285,31 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
     int64_t e = s;
     while (e < e_end) {
       const int nb = (int)mn64(UB, e_end - e);
-      int cc[UB];
+      Packed<T, NC> x[UB];
       float vv[UB];
-      float x[UB][NC];
 #pragma unroll
       for (int i = 0; i < UB; ++i) {
-        cc[i] = c[i];
         vv[i] = v[i];
-      }
-#pragma unroll
-      for (int i = 0; i < UB; ++i) {
-        if (i < nb) load_cols<NC>(Bb + (int64_t)cc[i] * A.ldb, lc, vec, x[i]);
+        if (i < nb && active) load_packed<NC>(Bb + (int64_t)c[i] * A.ldb, x[i]);
+        else zero_packed(x[i]);
       }
       const int64_t en = e + nb;
       if (en < e_end) load_batch(en, (int)mn64(UB, e_end - en));
+      if (en <= r_end) {  // the whole batch lies inside row r
 #pragma unroll
-      for (int i = 0; i < UB; ++i) {
-        if (i < nb) {
-          while (e + i >= r_end) {
-            finish(r);
-            ++r;
-            r_end = RP(r + 1);
+        for (int i = 0; i < UB; ++i)
+          if (i < nb) fma_row(vv[i], x[i], acc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < UB; ++i) {
+          if (i < nb) {
+            while (e + i >= r_end) {
+              finish(r);
+              ++r;
+              r_end = RP(r + 1);
+            }
+            fma_row(vv[i], x[i], acc);
           }
-#pragma unroll
-          for (int j = 0; j < NC; ++j) acc[j] = fmaf(vv[i], x[i][j], acc[j]);
         }
       }
       e = en;
@@ -273,38 +319,32 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
       link = false;
       while (r + 1 < A.rows && RP(r + 2) == e_end) {  // empty rows right after this range
         ++r;
-        store_cols<NC>(Cb + r * A.ldc, lc, vec, zero);
+        if (active) store_zero<NC>(Cb + r * A.ldc);
       }
     } else {
-      has_tail = true;
-#pragma unroll
-      for (int j = 0; j < NC; ++j) Tl[j] = acc[j];
+      has_tail = true;       // acc holds the open row's partial
       link = first && open;  // the whole range lies inside one row that started earlier
     }
   }
 
-  // Segmented inclusive scan of the workers' tail partials (segments = rows).
-  float S[NC];
+  // Segmented inclusive scan of the workers' tail partials (segments = rows); acc becomes
+  // the scanned value S.
 #pragma unroll
-  for (int j = 0; j < NC; ++j) S[j] = has_tail ? Tl[j] : 0.f;
+  for (int j = 0; j < NC; ++j) acc[j] = has_tail ? acc[j] : 0.f;
   int F = link ? 0 : 1;
 #pragma unroll
   for (int off = 1; off < WPW; off <<= 1) {
-    float Sp[NC];
-#pragma unroll
-    for (int j = 0; j < NC; ++j) Sp[j] = __shfl_up_sync(kFull, S[j], off * G);
     const int Fp = __shfl_up_sync(kFull, F, off * G);
-    if (g >= off) {
-      if (!F) {
 #pragma unroll
-        for (int j = 0; j < NC; ++j) S[j] += Sp[j];
-      }
-      F |= Fp;
+    for (int j = 0; j < NC; ++j) {
+      const float sp = __shfl_up_sync(kFull, acc[j], off * G);
+      if (g >= off && !F) acc[j] += sp;
     }
+    if (g >= off) F |= Fp;
   }
   if (g == WPW - 1) {
 #pragma unroll
-    for (int j = 0; j < NC; ++j) s_agg[wp][l * NC + j] = S[j];
+    for (int j = 0; j < NC; ++j) s_agg[wp][l * NC + j] = acc[j];
     if (l == 0) s_aggF[wp] = F;
   }
   __syncthreads();
@@ -316,28 +356,26 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
 #pragma unroll
     for (int j = 0; j < NC; ++j) inc[j] = fq ? s_agg[q][l * NC + j] : inc[j] + s_agg[q][l * NC + j];
   }
-  if (!F) {
 #pragma unroll
-    for (int j = 0; j < NC; ++j) S[j] += inc[j];
-  }
-  float E[NC];
-#pragma unroll
-  for (int j = 0; j < NC; ++j) E[j] = __shfl_up_sync(kFull, S[j], G);
-  if (g == 0) {
-#pragma unroll
-    for (int j = 0; j < NC; ++j) E[j] = inc[j];
+  for (int j = 0; j < NC; ++j) {
+    if (!F) acc[j] += inc[j];
+    float ej = __shfl_up_sync(kFull, acc[j], G);  // S of the previous worker
+    if (g == 0) ej = inc[j];
+    H[j] += ej;
   }
 
-  // Rows split across CTAs: write this CTA's partial, the last arrival combines.
+  // Rows split across CTAs (only rows longer than a part): write this CTA's partial; the
+  // last CTA to arrive sums all partials in part order and writes the row.
   auto cross_cta = [&](int64_t row, const float* val, bool row_ends_here) {
     const int64_t rs = RP(row), re = RP(row + 1);
     const int64_t P = A.P, nnz = A.nnz;
     const int64_t p1 = ((rs + 1) * P - 1) / nnz;  // part holding the row's first entry
     const int64_t pk = (re * P - 1) / nnz;        // part holding its last entry
     float* slot = (row_ends_here ? A.carry_head : A.carry_tail) + (int64_t)part * kCarryCols + n0;
+    if (active) {
 #pragma unroll
-    for (int j = 0; j < NC; ++j)
-      if (j < lc) slot[j] = val[j];
+      for (int j = 0; j < NC; ++j) slot[j] = val[j];
+    }
     __threadfence();
     __syncwarp(gmask);
     uint32_t* ctr = A.cnt + (int64_t)tile * P + p1;
@@ -349,37 +387,30 @@ __global__ void __launch_bounds__(kThreads) k_spmm_small(const SpmmArgs<T> A) {
       float sum[NC];
 #pragma unroll
       for (int j = 0; j < NC; ++j) sum[j] = 0.f;
-      for (int64_t q = p1; q < pk; ++q) {
-        const float* src = A.carry_tail + q * kCarryCols + n0;
+      if (active) {
+        for (int64_t q = p1; q < pk; ++q) {
+          const float* src = A.carry_tail + q * kCarryCols + n0;
 #pragma unroll
-        for (int j = 0; j < NC; ++j)
-          if (j < lc) sum[j] += __ldcg(src + j);
+          for (int j = 0; j < NC; ++j) sum[j] += __ldcg(src + j);
+        }
+        const float* src = A.carry_head + pk * kCarryCols + n0;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) sum[j] += __ldcg(src + j);
+        store_cols<NC>(Cb + row * A.ldc, sum);
       }
-      const float* src = A.carry_head + pk * kCarryCols + n0;
-#pragma unroll
-      for (int j = 0; j < NC; ++j)
-        if (j < lc) sum[j] += __ldcg(src + j);
-      store_cols<NC>(Cb + row * A.ldc, lc, vec, sum);
       if (l == 0) atomicExch(ctr, 0u);
     }
   };
 
   if (has_head) {
-    float val[NC];
-#pragma unroll
-    for (int j = 0; j < NC; ++j) val[j] = H[j] + E[j];
     if (h_row == ra && RP(ra) < a)
-      cross_cta(h_row, val, true);
-    else
-      store_cols<NC>(Cb + h_row * A.ldc, lc, vec, val);
+      cross_cta(h_row, H, true);
+    else if (active)
+      store_cols<NC>(Cb + h_row * A.ldc, H);
   }
-  if (w == NW - 1) {
-    int64_t lo = ra, hi = mn64(rb, A.rows - 1);  // row holding entry b - 1
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (RP(mid) <= b - 1) lo = mid; else hi = mid - 1;
-    }
-    if (RP(lo + 1) > b) cross_cta(lo, S, false);
+  if (w == NW - 1 && np > 0) {
+    const int64_t t = search_row(RP, ra, mn64(rb, A.rows - 1), b - 1);  // row holding entry b - 1
+    if (RP(t + 1) > b) cross_cta(t, acc, false);
   }
 }
 
@@ -389,102 +420,123 @@ template <typename T>
 struct SddmmArgs {
   const int32_t* row_ptr;
   const int32_t* col;
-  const int32_t* part_nnz;
-  const int32_t* part_row;
-  const T* X;   // K x N
-  const T* dY;  // M x N
-  T* dW;        // [nnz]
+  const int4* desc;  // [P] per-CTA work descriptors (forward ones)
+  const T* X;        // K x N
+  const T* dY;       // M x N
+  T* dW;             // [nnz]
   int64_t ldx, lddy;
   int64_t rows;
   int64_t nnz;
-  int N;
-  int vec;
+  int N;             // a multiple of NC
 };
 
+template <typename T, int NC>
+__device__ __forceinline__ float dot_packed(const Packed<T, NC>& x, const Packed<T, NC>& y, float d) {
+  if constexpr (NC == 1) {
+    return fmaf(unpack<T, NC>(x, 0), unpack<T, NC>(y, 0), d);
+  } else {
+    float2 d2 = make_float2(d, 0.f);
+#pragma unroll
+    for (int j = 0; j < NC; j += 2)
+      d2 = __ffma2_rn(make_float2(unpack<T, NC>(x, j), unpack<T, NC>(x, j + 1)),
+                      make_float2(unpack<T, NC>(y, j), unpack<T, NC>(y, j + 1)), d2);
+    return d2.x + d2.y;
+  }
+}
+
 template <typename T, int NC, int G>
-__global__ void __launch_bounds__(kThreads) k_sddmm_small(const SddmmArgs<T> A) {
+__global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> A) {
   constexpr int NW = kThreads / G;
   constexpr int NT = NC * G;
-  constexpr int UB = NC >= 8 ? 4 : 8;
+  constexpr int UB = sddmm_batch<T, NC>();
   __shared__ int32_t s_rp[kRowCap];
+  __shared__ float s_dw[kStageCap];
 
+  pdl_launch_dependents();
   const int part = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31;
   const int w = tid / G, l = tid % G;
   const int lane_base = lane - l;
   const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
+  pdl_wait();
 
-  const int64_t a = A.part_nnz[part], b = A.part_nnz[part + 1];
+  const int4 dsc = __ldg(A.desc + part);
+  const int64_t a = dsc.x, b = dsc.y, ra = dsc.z, rb = dsc.w;
   const int64_t np = b - a;
+  const bool staged = np <= kStageCap;
   const int64_t s = a + (np * w) / NW;
   const int64_t e_end = a + (np * (w + 1)) / NW;
-  const int64_t ra = A.part_row[part];
-  const int64_t rb = A.part_row[part + 1];
+  int c[UB];
+  auto load_batch = [&](int64_t e0, int nb) {
+#pragma unroll
+    for (int i = 0; i < UB; ++i)
+      if (i < nb) c[i] = __ldg(A.col + e0 + i);
+  };
+  if (s < e_end) load_batch(s, (int)mn64(UB, e_end - s));
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
-  const bool in_smem = span <= kRowCap;
+  const bool in_smem = np > 0 && span <= kRowCap;
   if (in_smem)
     for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.row_ptr + ra + i);
   __syncthreads();
   auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.row_ptr + r); };
-  if (s >= e_end) return;
-  const bool vec = A.vec != 0;
 
-  int64_t lo = ra, hi = mn64(rb, A.rows - 1);
-  while (lo < hi) {
-    const int64_t mid = (lo + hi + 1) >> 1;
-    if (RP(mid) <= s) lo = mid; else hi = mid - 1;
+  if (s < e_end) {
+    int64_t r = search_row(RP, ra, mn64(rb, A.rows - 1), s);
+    int64_t r_end = RP(r + 1);
+    for (int64_t e = s; e < e_end; e += UB) {
+      const int nb = (int)mn64(UB, e_end - e);
+      int cc[UB];
+      int rr[UB];
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+        cc[i] = c[i];
+        rr[i] = (int)r;
+        if (i < nb) {
+          while (e + i >= r_end) {
+            ++r;
+            r_end = RP(r + 1);
+          }
+          rr[i] = (int)r;
+        }
+      }
+      const int64_t en = e + nb;
+      if (en < e_end) load_batch(en, (int)mn64(UB, e_end - en));
+      float d[UB];
+#pragma unroll
+      for (int i = 0; i < UB; ++i) d[i] = 0.f;
+      for (int n0 = l * NC; n0 < A.N; n0 += NT) {
+        Packed<T, NC> xv[UB], yv[UB];
+#pragma unroll
+        for (int i = 0; i < UB; ++i) {
+          if (i < nb) {
+            load_packed<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, xv[i]);
+            load_packed<NC>(A.dY + (int64_t)rr[i] * A.lddy + n0, yv[i]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < UB; ++i)
+          if (i < nb) d[i] = dot_packed(xv[i], yv[i], d[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < UB; ++i) {
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) d[i] += __shfl_xor_sync(gmask, d[i], off);
+      }
+      if (l == 0) {
+#pragma unroll
+        for (int i = 0; i < UB; ++i) {
+          if (i < nb) {
+            if (staged) s_dw[e + i - a] = d[i];
+            else store1(A.dW + e + i, d[i]);
+          }
+        }
+      }
+    }
   }
-  int64_t r = lo;
-  int64_t r_end = RP(r + 1);
-  for (int64_t e = s; e < e_end; e += UB) {
-    const int nb = (int)mn64(UB, e_end - e);
-    int cc[UB];
-    int64_t rr[UB];
-#pragma unroll
-    for (int i = 0; i < UB; ++i) {
-      cc[i] = 0;
-      rr[i] = r;
-      if (i < nb) {
-        cc[i] = __ldg(A.col + e + i);
-        while (e + i >= r_end) {
-          ++r;
-          r_end = RP(r + 1);
-        }
-        rr[i] = r;
-      }
-    }
-    float d[UB];
-#pragma unroll
-    for (int i = 0; i < UB; ++i) d[i] = 0.f;
-    for (int n0 = l * NC; n0 < A.N; n0 += NT) {
-      const int lc = min(NC, A.N - n0);
-      float xv[UB][NC], yv[UB][NC];
-#pragma unroll
-      for (int i = 0; i < UB; ++i) {
-        if (i < nb) {
-          load_cols<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, lc, vec, xv[i]);
-          load_cols<NC>(A.dY + rr[i] * A.lddy + n0, lc, vec, yv[i]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < UB; ++i) {
-        if (i < nb) {
-#pragma unroll
-          for (int j = 0; j < NC; ++j) d[i] = fmaf(xv[i][j], yv[i][j], d[i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < UB; ++i) {
-#pragma unroll
-      for (int off = G / 2; off > 0; off >>= 1) d[i] += __shfl_xor_sync(gmask, d[i], off);
-    }
-    if (l == 0) {
-#pragma unroll
-      for (int i = 0; i < UB; ++i)
-        if (i < nb) store1(A.dW + e + i, d[i]);
-    }
+  if (staged) {  // coalesced write-out of the CTA's range
+    __syncthreads();
+    for (int64_t i = tid; i < np; i += kThreads) store1(A.dW + a + i, s_dw[i]);
   }
 }
 
@@ -509,9 +561,33 @@ bool aligned(const void* p, int64_t ld, int nc, int elem) {
   return ((uintptr_t)p % (uintptr_t)(nc * elem)) == 0 && (ld % nc) == 0;
 }
 
+// Widest vector (<= 16 bytes) that divides `ncols` and keeps every listed row aligned.
+int pick_nc(int ncols, int elem, const void* p0, int64_t ld0, const void* p1, int64_t ld1) {
+  int nc = 16 / elem;
+  while (nc > 1 && !((ncols % nc) == 0 && aligned(p0, ld0, nc, elem) && aligned(p1, ld1, nc, elem))) nc >>= 1;
+  return nc;
+}
+
+template <typename Args>
+cudaError_t launch_pdl(void (*kern)(const Args), dim3 grid, cudaStream_t s, const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args);
+}
+
 template <typename T, bool TRANS>
 using SpmmKernel = void (*)(const SpmmArgs<T>);
 
+// Instantiated shapes: NC = 16 bytes' worth of elements with G = 1..8 (bf16) / 1..16
+// (fp32) lanes, narrower vectors with one lane, and scalars with G = 1..32.
 template <typename T, bool TRANS>
 SpmmKernel<T, TRANS> pick_spmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
@@ -556,18 +632,12 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     const int ncols = (int)std::min<int64_t>(kCarryCols, N - col0);
     const T* Bc = B + col0;
     T* Cc = C + col0;
-    const int ncmax = 16 / elem;
-    int nc = std::min(ncmax, pow2ceil(ncols));
-    while (nc > 1 && !(aligned(Bc, ldb, nc, elem) && aligned(Cc, ldc, nc, elem))) nc >>= 1;
+    int nc = pick_nc(ncols, elem, Bc, ldb, Cc, ldc);
     int g = pow2ceil((ncols + nc - 1) / nc);
-    if (nc > 1) {
-      // wide vectors: the instantiated worker widths
-      const int gmax = (elem == 2) ? (nc == 8 ? 8 : 1) : (nc == 4 ? 16 : 1);
-      if (g > gmax) {
-        // fall back to narrower vectors with more lanes
-        nc = 1;
-        g = pow2ceil(ncols);
-      }
+    const int gmax = nc == 1 ? 32 : (elem == 2 ? (nc == 8 ? 8 : 1) : (nc == 4 ? 16 : 1));
+    if (g > gmax) {  // narrow vectors come with one lane only: use scalars instead
+      nc = 1;
+      g = pow2ceil(ncols);
     }
     g = std::min(g, 32);
     const int nt = nc * g;
@@ -579,8 +649,7 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     A.idx = TRANS ? L->csc_row : L->col;
     A.perm = TRANS ? L->perm : nullptr;
     A.vals = values;
-    A.part_nnz = TRANS ? L->part_nnz_t : L->part_nnz;
-    A.part_row = TRANS ? L->part_col : L->part_row;
+    A.desc = TRANS ? L->desc_t : L->desc_f;
     A.B = Bc;
     A.C = Cc;
     A.ldb = ldb;
@@ -589,12 +658,10 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     A.nnz = L->nnz;
     A.P = L->P;
     A.ncols = ncols;
-    A.vec = nc > 1 ? 1 : 0;
     A.carry_tail = TRANS ? L->carry_tail_b : L->carry_tail_f;
     A.carry_head = TRANS ? L->carry_head_b : L->carry_head_f;
     A.cnt = TRANS ? L->cnt_b : L->cnt_f;
-    kern<<<dim3((unsigned)L->P, (unsigned)tiles), kThreads, 0, s>>>(A);
-    SNK_CUDA_TRY(cudaGetLastError());
+    SNK_CUDA_TRY(launch_pdl(kern, dim3((unsigned)L->P, (unsigned)tiles), s, A));
   }
   return SNK_OK;
 }
@@ -603,22 +670,20 @@ template <typename T>
 snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* X, int64_t ldx, int64_t N, T* dW,
                        cudaStream_t s) {
   const int elem = (int)sizeof(T);
-  const int ncmax = 16 / elem;
-  int nc = std::min<int64_t>(ncmax, pow2ceil((int)std::min<int64_t>(N, 1 << 20)));
-  while (nc > 1 && !(aligned(X, ldx, nc, elem) && aligned(dY, lddy, nc, elem))) nc >>= 1;
+  const int ncap = (int)std::min<int64_t>(N, 1 << 20);
+  int nc = pick_nc(std::max(ncap, 1), elem, X, ldx, dY, lddy);
   int g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>((N + nc - 1) / nc, 64)));
   auto kern = pick_sddmm<T>(nc, g);
   if (kern == nullptr) {
     nc = 1;
-    g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>(N, 64)));
+    g = (int)std::min<int64_t>(32, pow2ceil((int)std::max<int64_t>(1, std::min<int64_t>(N, 64))));
     kern = pick_sddmm<T>(nc, g);
   }
   if (kern == nullptr) return SNK_ERR_UNSUPPORTED;
   SddmmArgs<T> A;
   A.row_ptr = L->row_ptr;
   A.col = L->col;
-  A.part_nnz = L->part_nnz;
-  A.part_row = L->part_row;
+  A.desc = L->desc_f;
   A.X = X;
   A.dY = dY;
   A.dW = dW;
@@ -627,9 +692,7 @@ snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* 
   A.rows = L->M;
   A.nnz = L->nnz;
   A.N = (int)N;
-  A.vec = nc > 1 ? 1 : 0;
-  kern<<<(unsigned)L->P, kThreads, 0, s>>>(A);
-  SNK_CUDA_TRY(cudaGetLastError());
+  SNK_CUDA_TRY(launch_pdl(kern, dim3((unsigned)L->P), s, A));
   return SNK_OK;
 }
 

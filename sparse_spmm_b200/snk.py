@@ -197,9 +197,12 @@ class Layout:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            snk_destroy(h)
-            self.handle = None
+        if h and _lib is not None:
+            try:
+                _lib.snk_destroy(h)
+            except Exception:  # interpreter shutdown: the library may already be gone
+                pass
+        self.handle = None
 
     def close(self):
         self.__del__()

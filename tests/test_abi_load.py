@@ -48,8 +48,8 @@ def test_default_num_parts(lib):
     assert snk.snk_default_num_parts(0, 148) == 1
     assert snk.snk_default_num_parts(256, 148) == 1
     assert snk.snk_default_num_parts(257, 148) == 2
-    assert snk.snk_default_num_parts(838861, 148) == 592
-    assert snk.snk_default_num_parts(10**9, 148) == 592
+    assert snk.snk_default_num_parts(838861, 148) == 444
+    assert snk.snk_default_num_parts(10**9, 148) == 444
 
 
 def test_workspace_bytes_rejects_bad_sizes(lib):
