@@ -164,6 +164,30 @@ SNK_API snk_status snk_backward_weight(const snk_layout* L, const void* dY, int6
 SNK_API snk_status snk_restructure(snk_layout* L, void* values, int64_t drop_count, uint64_t seed,
                            float regrow_value, int32_t* old_to_new, snk_stream stream);
 
+/*
+ * snk_csr_forward_static -- Y = W X straight from a CSR matrix, allocating nothing.
+ * (This entry point is the library's own addition; the paper has no counterpart.)
+ * For callers that cannot allocate device memory at all -- e.g. code given a CSR matrix
+ * and its activation buffers by a host framework that owns every allocation -- and so
+ * cannot provide the workspace that snk_build needs.  The kernel's scratch (work
+ * descriptors, carry slots of rows split between CTAs and their arrival counters) lives
+ * in a fixed static device array of about 0.4 MB that every GPU loading the library holds
+ * until process exit; at most SNK_STATIC_MAX_PARTS CTAs use it per launch.
+ * row_ptr: int32 [M+1] (row_ptr[0] = 0, non-decreasing, row_ptr[M] = nnz); col: int32
+ * [nnz] in [0, K); values: [nnz] of dt.  The arrays are NOT validated: an index outside
+ * its range is undefined behaviour.  X: K x N (ldx >= N); Y: M x N (ldy >= N),
+ * overwritten.  num_parts: 0 = the default split, else 1..SNK_STATIC_MAX_PARTS (larger
+ * values return SNK_ERR_UNSUPPORTED).  Calls no allocator.  The first call on a device
+ * looks up the scratch array's device address, so make it before any stream capture on
+ * that device.  Every call shares the one scratch array (counters are cleared at the
+ * start of each call): calls that overlap on the GPU, on any stream, race.
+ */
+#define SNK_STATIC_MAX_PARTS 512
+SNK_API snk_status snk_csr_forward_static(int64_t M, int64_t K, int64_t nnz, const int32_t* row_ptr,
+                                          const int32_t* col, const void* values, snk_dtype dt, const void* X,
+                                          int64_t N, int64_t ldx, void* Y, int64_t ldy, int32_t num_parts,
+                                          snk_stream stream);
+
 /* Fill *v with the layout's sizes and device pointers.  Returns SNK_ERR_INVALID_ARG for
  * NULL arguments. */
 SNK_API snk_status snk_layout_info(const snk_layout* L, snk_layout_view* v);

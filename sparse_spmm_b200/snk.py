@@ -166,6 +166,19 @@ def snk_destroy(handle):
         load_library().snk_destroy(handle)
 
 
+def snk_csr_forward_static(M, K, row_ptr, col, values, X, Y, num_parts=0, stream=None):
+    """Y = W X from a plain CSR matrix; the library allocates nothing (static scratch)."""
+    lib = load_library()
+    fn = lib.snk_csr_forward_static
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p]
+    N = X.shape[1]
+    _check(fn(M, K, col.numel(), _ptr(row_ptr), _ptr(col), _ptr(values), _dtype_code(X.dtype), _ptr(X), N,
+              _ld(X), _ptr(Y), _ld(Y), num_parts, _stream(stream)), "snk_csr_forward_static")
+
+
 # ----------------------------------------------------------------------------- convenience
 
 class Layout:
