@@ -192,8 +192,10 @@ __global__ void __launch_bounds__(kScanThreads) k_tile_sums(const uint32_t* __re
   if (threadIdx.x == 0) sums[blockIdx.x] = tot;
 }
 
-__global__ void __launch_bounds__(kScanThreads) k_tile_scan(const uint32_t* __restrict__ a, uint32_t* __restrict__ out,
-                                                            int64_t n, const uint32_t* __restrict__ offs) {
+// May run in place (out == a): every thread reads its items before the block scan's
+// barriers and writes them after.
+__global__ void __launch_bounds__(kScanThreads) k_tile_scan(const uint32_t* a, uint32_t* out, int64_t n,
+                                                            const uint32_t* __restrict__ offs) {
   __shared__ uint32_t wt[32];
   const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanItems;
   uint32_t x[kScanItems];
@@ -475,9 +477,14 @@ snk_status radix_sort(snk_layout* L, int64_t n, int nbits, cudaStream_t s, bool*
   uint32_t* vo = L->vals1;
   if (n > 0) {
     const int nblocks = (int)ceil_div(n, kSortTile);
+    const int64_t nh = (int64_t)256 * nblocks;
+    const int64_t nt = ceil_div(nh, kScanTile);
     for (int shift = 0; shift < nbits; shift += 8) {
       k_rs_hist<<<nblocks, kSortThreads, 0, s>>>(ki, n, shift, L->hist, nblocks);
-      k_scan_single<<<1, kScanThreads, 0, s>>>(L->hist, (int64_t)256 * nblocks, nullptr);
+      // exclusive scan of the digit-major histogram, in place (tile sums, their scan, tiles)
+      k_tile_sums<<<(unsigned)nt, kScanThreads, 0, s>>>(L->hist, nh, L->scan_tmp);
+      k_scan_single<<<1, kScanThreads, 0, s>>>(L->scan_tmp, nt, nullptr);
+      k_tile_scan<<<(unsigned)nt, kScanThreads, 0, s>>>(L->hist, L->hist, nh, L->scan_tmp);
       k_rs_scatter<<<nblocks, kSortThreads, 0, s>>>(ki, vi, ko, vo, n, shift, L->hist, nblocks);
       std::swap(ki, ko);
       std::swap(vi, vo);
@@ -561,7 +568,7 @@ size_t carve(snk_layout* L, uint8_t* base) {
   L->flags2 = c.take<uint32_t>(L->scap);
   L->grown = c.take<uint64_t>(nnz);
   L->vcopy = c.take<uint8_t>(4 * nnz);
-  L->scan_tmp = c.take<uint32_t>(ceil_div(L->scap, kScanTile) + 64);
+  L->scan_tmp = c.take<uint32_t>(ceil_div(L->scap, kScanTile) + ceil_div((int64_t)256 * ceil_div(L->scap, kSortTile), kScanTile) + 64);
   return c.off;
 }
 

@@ -22,6 +22,8 @@
 //
 // Gathered rows of the dense operand are kept packed (bf16 pairs in 32-bit words) until
 // the FMA and are multiplied with packed fp32 FMAs (two lanes of fp32 per instruction).
+// A lane holds up to 32 bytes of a row (two 16-byte vector loads), so few lanes repeat
+// the per-entry index and value loads.
 #include <algorithm>
 
 #include "internal.cuh"
@@ -49,7 +51,8 @@ __device__ __forceinline__ void store1(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
 // NC consecutive elements of T held as loaded: 32-bit words (two bf16 per word, or one
-// float).  NC > 1 loads are single aligned vector loads (the host guarantees alignment).
+// float).  Groups of more than one element are loaded with aligned vector loads of up to
+// 16 bytes each (the host guarantees 16-byte alignment of every row start and column).
 template <typename T, int NC>
 struct Packed {
   static constexpr int W = sizeof(T) == 2 ? (NC + 1) / 2 : NC;
@@ -58,28 +61,20 @@ struct Packed {
 
 template <int NC, typename T>
 __device__ __forceinline__ void load_packed(const T* p, Packed<T, NC>& r) {
-  if constexpr (sizeof(T) == 2) {
-    if constexpr (NC == 8) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-      r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
-    } else if constexpr (NC == 4) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      r.w[0] = v.x; r.w[1] = v.y;
-    } else if constexpr (NC == 2) {
-      r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
-    } else {
-      r.w[0] = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16;  // one value, high half
+  constexpr int W = Packed<T, NC>::W;
+  if constexpr (W >= 4) {
+#pragma unroll
+    for (int k = 0; k < W; k += 4) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + k / 4);
+      r.w[k] = v.x; r.w[k + 1] = v.y; r.w[k + 2] = v.z; r.w[k + 3] = v.w;
     }
+  } else if constexpr (W == 2) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    r.w[0] = v.x; r.w[1] = v.y;
+  } else if constexpr (sizeof(T) == 2 && NC == 1) {
+    r.w[0] = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16;  // one value, high half
   } else {
-    if constexpr (NC == 4) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-      r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
-    } else if constexpr (NC == 2) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      r.w[0] = v.x; r.w[1] = v.y;
-    } else {
-      r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
-    }
+    r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
   }
 }
 
@@ -122,13 +117,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Store NC values (rounded once to T).  NC > 1 stores are single aligned vector stores.
+// Store NC values (rounded once to T) with aligned vector stores of up to 16 bytes.
 template <int NC, typename T>
 __device__ __forceinline__ void store_cols(T* p, const float* v) {
   if constexpr (sizeof(T) == 2) {
-    if constexpr (NC == 8) {
-      *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                                pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    if constexpr (NC >= 8) {
+#pragma unroll
+      for (int k = 0; k < NC; k += 8)
+        reinterpret_cast<uint4*>(p)[k / 8] = make_uint4(pack_bf16x2(v[k], v[k + 1]), pack_bf16x2(v[k + 2], v[k + 3]),
+                                                        pack_bf16x2(v[k + 4], v[k + 5]), pack_bf16x2(v[k + 6], v[k + 7]));
     } else if constexpr (NC == 4) {
       *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
     } else if constexpr (NC == 2) {
@@ -137,8 +134,10 @@ __device__ __forceinline__ void store_cols(T* p, const float* v) {
       store1(p, v[0]);
     }
   } else {
-    if constexpr (NC == 4) {
-      *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    if constexpr (NC >= 4) {
+#pragma unroll
+      for (int k = 0; k < NC; k += 4)
+        reinterpret_cast<float4*>(p)[k / 4] = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
     } else if constexpr (NC == 2) {
       *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
     } else {
@@ -189,6 +188,7 @@ struct SpmmArgs {
   int64_t nnz;
   int P;
   int ncols;           // columns in this launch (<= kCarryCols, a multiple of NC)
+  int b32;             // every gathered row offset c * ldb fits in 32 bits
   float* carry_tail;   // [P][kCarryCols]
   float* carry_head;   // [P][kCarryCols]
   uint32_t* cnt;       // [kMaxTiles][P], zero between launches
@@ -196,9 +196,9 @@ struct SpmmArgs {
 
 // Entries in flight per worker: as many as the register budget of 3 CTAs per SM allows.
 template <typename T, int NC>
-constexpr int spmm_batch() { return NC * (int)sizeof(T) >= 16 ? 4 : 8; }
+constexpr int spmm_batch() { return NC * (int)sizeof(T) >= 32 ? 3 : (NC * (int)sizeof(T) >= 16 ? 6 : 8); }
 template <typename T, int NC>
-constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 8 ? 4 : 6; }
+constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 32 ? 2 : (NC * (int)sizeof(T) >= 8 ? 4 : 6); }
 
 template <typename T, int NC, int G, bool TRANS>
 __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A) {
@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   __shared__ int32_t s_rp[kRowCap];
   __shared__ float s_agg[NWARPS][NT];
   __shared__ int s_aggF[NWARPS];
+  __shared__ float s_head[NC][kThreads];  // the worker's first, still open row (per lane)
 
   pdl_launch_dependents();
   const int part = blockIdx.x, tile = blockIdx.y;
@@ -223,25 +224,27 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
 
   const int4 dsc = __ldg(A.desc + part);
   const int64_t a = dsc.x, b = dsc.y, ra = dsc.z, rb = dsc.w;
-  const int64_t np = b - a;
-  const int64_t s = a + (np * w) / NW;
-  const int64_t e_end = a + (np * (w + 1)) / NW;
+  const int np = (int)(b - a);
+  // the worker's piece, as offsets from a
+  const int s = (int)(((int64_t)np * w) / NW);
+  const int e_end = (int)(((int64_t)np * (w + 1)) / NW);
+  const int32_t* __restrict__ idx = A.idx + a;
+  const int32_t* __restrict__ prm = TRANS ? A.perm + a : nullptr;
+  const T* __restrict__ vals = TRANS ? A.vals : A.vals + a;
 
   // the worker's next batch of indices / values (prefetched one batch ahead)
   int c[UB];
   float v[UB];
-  auto load_batch = [&](int64_t e0, int nb) {
+  auto load_batch = [&](int e0, int nb) {
 #pragma unroll
     for (int i = 0; i < UB; ++i) {
       if (i < nb) {
-        const int64_t j = e0 + i;
-        c[i] = __ldg(A.idx + j);
-        const int64_t pe = TRANS ? (int64_t)__ldg(A.perm + j) : j;
-        v[i] = load1(A.vals + pe);
+        c[i] = __ldg(idx + e0 + i);
+        v[i] = TRANS ? load1(vals + __ldg(prm + e0 + i)) : load1(vals + e0 + i);
       }
     }
   };
-  if (s < e_end) load_batch(s, (int)mn64(UB, e_end - s));
+  if (s < e_end) load_batch(s, min(UB, e_end - s));
 
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
@@ -249,22 +252,25 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   if (in_smem)
     for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.ptr + ra + i);
   __syncthreads();
-  auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.ptr + r); };
+  // row pointers, relative to a
+  auto RP = [&](int64_t r) -> int { return (in_smem ? s_rp[r - ra] : __ldg(A.ptr + r)) - (int)a; };
 
   const T* __restrict__ Bb = A.B + n0;
   T* __restrict__ Cb = A.C + n0;
+  const unsigned ldb = (unsigned)A.ldb;
+  const bool small_b = A.b32 != 0;
 
-  float acc[NC], H[NC];
+  float acc[NC];
 #pragma unroll
-  for (int j = 0; j < NC; ++j) acc[j] = H[j] = 0.f;
+  for (int j = 0; j < NC; ++j) acc[j] = 0.f;
   bool has_head = false, has_tail = false, link = true;
   int64_t h_row = -1;
 
   if (s < e_end) {
-    int64_t r = search_row(RP, ra, mn64(rb, A.rows - 1), s);
-    int64_t r_end = RP(r + 1);
+    int64_t r = search_row([&](int64_t q) { return (int64_t)RP(q); }, ra, mn64(rb, A.rows - 1), s);
+    int r_end = RP(r + 1);
     bool first = true, open = RP(r) < s;
-    if (s == 0 && active)  // empty rows ahead of the first entry
+    if (s == 0 && a == 0 && active)  // empty rows ahead of the first entry
       for (int64_t q = 0; q < r; ++q) store_zero<NC>(Cb + q * A.ldc);
 
     auto finish = [&](int64_t row) {
@@ -272,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
         has_head = true;
         h_row = row;
 #pragma unroll
-        for (int j = 0; j < NC; ++j) H[j] = acc[j];
+        for (int j = 0; j < NC; ++j) s_head[j][tid] = acc[j];
       } else if (active) {
         store_cols<NC>(Cb + row * A.ldc, acc);
       }
@@ -282,19 +288,23 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
       for (int j = 0; j < NC; ++j) acc[j] = 0.f;
     };
 
-    int64_t e = s;
+    int e = s;
     while (e < e_end) {
-      const int nb = (int)mn64(UB, e_end - e);
+      const int nb = min(UB, e_end - e);
       Packed<T, NC> x[UB];
       float vv[UB];
 #pragma unroll
       for (int i = 0; i < UB; ++i) {
         vv[i] = v[i];
-        if (i < nb && active) load_packed<NC>(Bb + (int64_t)c[i] * A.ldb, x[i]);
-        else zero_packed(x[i]);
+        if (i < nb && active) {
+          const T* src = small_b ? Bb + (unsigned)c[i] * ldb : Bb + (int64_t)c[i] * A.ldb;
+          load_packed<NC>(src, x[i]);
+        } else {
+          zero_packed(x[i]);
+        }
       }
-      const int64_t en = e + nb;
-      if (en < e_end) load_batch(en, (int)mn64(UB, e_end - en));
+      const int en = e + nb;
+      if (en < e_end) load_batch(en, min(UB, e_end - en));
       if (en <= r_end) {  // the whole batch lies inside row r
 #pragma unroll
         for (int i = 0; i < UB; ++i)
@@ -348,26 +358,27 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
     if (l == 0) s_aggF[wp] = F;
   }
   __syncthreads();
-  float inc[NC];
+  float H[NC];
 #pragma unroll
-  for (int j = 0; j < NC; ++j) inc[j] = 0.f;
+  for (int j = 0; j < NC; ++j) H[j] = 0.f;  // holds the incoming prefix until it is added
   for (int q = 0; q < wp; ++q) {
     const int fq = s_aggF[q];
 #pragma unroll
-    for (int j = 0; j < NC; ++j) inc[j] = fq ? s_agg[q][l * NC + j] : inc[j] + s_agg[q][l * NC + j];
+    for (int j = 0; j < NC; ++j) H[j] = fq ? s_agg[q][l * NC + j] : H[j] + s_agg[q][l * NC + j];
   }
 #pragma unroll
   for (int j = 0; j < NC; ++j) {
-    if (!F) acc[j] += inc[j];
+    const float inc = H[j];
+    if (!F) acc[j] += inc;
     float ej = __shfl_up_sync(kFull, acc[j], G);  // S of the previous worker
-    if (g == 0) ej = inc[j];
-    H[j] += ej;
+    if (g == 0) ej = inc;
+    H[j] = has_head ? s_head[j][tid] + ej : 0.f;
   }
 
   // Rows split across CTAs (only rows longer than a part): write this CTA's partial; the
   // last CTA to arrive sums all partials in part order and writes the row.
   auto cross_cta = [&](int64_t row, const float* val, bool row_ends_here) {
-    const int64_t rs = RP(row), re = RP(row + 1);
+    const int64_t rs = (int64_t)RP(row) + a, re = (int64_t)RP(row + 1) + a;
     const int64_t P = A.P, nnz = A.nnz;
     const int64_t p1 = ((rs + 1) * P - 1) / nnz;  // part holding the row's first entry
     const int64_t pk = (re * P - 1) / nnz;        // part holding its last entry
@@ -403,14 +414,14 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   };
 
   if (has_head) {
-    if (h_row == ra && RP(ra) < a)
+    if (h_row == ra && RP(ra) < 0)
       cross_cta(h_row, H, true);
     else if (active)
       store_cols<NC>(Cb + h_row * A.ldc, H);
   }
   if (w == NW - 1 && np > 0) {
-    const int64_t t = search_row(RP, ra, mn64(rb, A.rows - 1), b - 1);  // row holding entry b - 1
-    if (RP(t + 1) > b) cross_cta(t, acc, false);
+    const int64_t t = search_row([&](int64_t q) { return (int64_t)RP(q); }, ra, mn64(rb, A.rows - 1), np - 1);
+    if (RP(t + 1) > np) cross_cta(t, acc, false);
   }
 }
 
@@ -462,37 +473,39 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
 
   const int4 dsc = __ldg(A.desc + part);
   const int64_t a = dsc.x, b = dsc.y, ra = dsc.z, rb = dsc.w;
-  const int64_t np = b - a;
+  const int np = (int)(b - a);
   const bool staged = np <= kStageCap;
-  const int64_t s = a + (np * w) / NW;
-  const int64_t e_end = a + (np * (w + 1)) / NW;
+  const int s = (int)(((int64_t)np * w) / NW);
+  const int e_end = (int)(((int64_t)np * (w + 1)) / NW);
+  const int32_t* __restrict__ col = A.col + a;
   int c[UB];
-  auto load_batch = [&](int64_t e0, int nb) {
+  auto load_batch = [&](int e0, int nb) {
 #pragma unroll
     for (int i = 0; i < UB; ++i)
-      if (i < nb) c[i] = __ldg(A.col + e0 + i);
+      if (i < nb) c[i] = __ldg(col + e0 + i);
   };
-  if (s < e_end) load_batch(s, (int)mn64(UB, e_end - s));
+  if (s < e_end) load_batch(s, min(UB, e_end - s));
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
   const bool in_smem = np > 0 && span <= kRowCap;
   if (in_smem)
     for (int64_t i = tid; i < span; i += kThreads) s_rp[i] = __ldg(A.row_ptr + ra + i);
   __syncthreads();
-  auto RP = [&](int64_t r) -> int64_t { return in_smem ? (int64_t)s_rp[r - ra] : (int64_t)__ldg(A.row_ptr + r); };
+  auto RP = [&](int64_t r) -> int { return (in_smem ? s_rp[r - ra] : __ldg(A.row_ptr + r)) - (int)a; };
 
   if (s < e_end) {
-    int64_t r = search_row(RP, ra, mn64(rb, A.rows - 1), s);
-    int64_t r_end = RP(r + 1);
-    for (int64_t e = s; e < e_end; e += UB) {
-      const int nb = (int)mn64(UB, e_end - e);
+    int64_t r = search_row([&](int64_t q) { return (int64_t)RP(q); }, ra, mn64(rb, A.rows - 1), s);
+    int r_end = RP(r + 1);
+    for (int e = s; e < e_end; e += UB) {
+      const int nb = min(UB, e_end - e);
       int cc[UB];
       int rr[UB];
+      const bool one_row = e + nb <= r_end;  // the whole batch lies inside row r
 #pragma unroll
       for (int i = 0; i < UB; ++i) {
         cc[i] = c[i];
         rr[i] = (int)r;
-        if (i < nb) {
+        if (!one_row && i < nb) {
           while (e + i >= r_end) {
             ++r;
             r_end = RP(r + 1);
@@ -500,23 +513,32 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
           rr[i] = (int)r;
         }
       }
-      const int64_t en = e + nb;
-      if (en < e_end) load_batch(en, (int)mn64(UB, e_end - en));
+      const int en = e + nb;
+      if (en < e_end) load_batch(en, min(UB, e_end - en));
       float d[UB];
 #pragma unroll
       for (int i = 0; i < UB; ++i) d[i] = 0.f;
       for (int n0 = l * NC; n0 < A.N; n0 += NT) {
-        Packed<T, NC> xv[UB], yv[UB];
-#pragma unroll
-        for (int i = 0; i < UB; ++i) {
-          if (i < nb) {
-            load_packed<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, xv[i]);
-            load_packed<NC>(A.dY + (int64_t)rr[i] * A.lddy + n0, yv[i]);
-          }
-        }
+        Packed<T, NC> xv[UB];
 #pragma unroll
         for (int i = 0; i < UB; ++i)
-          if (i < nb) d[i] = dot_packed(xv[i], yv[i], d[i]);
+          if (i < nb) load_packed<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, xv[i]);
+        if (one_row) {
+          Packed<T, NC> yv;
+          load_packed<NC>(A.dY + (int64_t)rr[0] * A.lddy + n0, yv);
+#pragma unroll
+          for (int i = 0; i < UB; ++i)
+            if (i < nb) d[i] = dot_packed(xv[i], yv, d[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < UB; ++i) {
+            if (i < nb) {
+              Packed<T, NC> yv;
+              load_packed<NC>(A.dY + (int64_t)rr[i] * A.lddy + n0, yv);
+              d[i] = dot_packed(xv[i], yv, d[i]);
+            }
+          }
+        }
       }
 #pragma unroll
       for (int i = 0; i < UB; ++i) {
@@ -527,8 +549,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
 #pragma unroll
         for (int i = 0; i < UB; ++i) {
           if (i < nb) {
-            if (staged) s_dw[e + i - a] = d[i];
-            else store1(A.dW + e + i, d[i]);
+            if (staged) s_dw[e + i] = d[i];
+            else store1(A.dW + a + e + i, d[i]);
           }
         }
       }
@@ -536,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
   }
   if (staged) {  // coalesced write-out of the CTA's range
     __syncthreads();
-    for (int64_t i = tid; i < np; i += kThreads) store1(A.dW + a + i, s_dw[i]);
+    for (int i = tid; i < np; i += kThreads) store1(A.dW + a + i, s_dw[i]);
   }
 }
 
@@ -561,10 +583,15 @@ bool aligned(const void* p, int64_t ld, int nc, int elem) {
   return ((uintptr_t)p % (uintptr_t)(nc * elem)) == 0 && (ld % nc) == 0;
 }
 
-// Widest vector (<= 16 bytes) that divides `ncols` and keeps every listed row aligned.
+// Widest per-lane group (<= 32 bytes, in vectors of <= 16 bytes) that divides `ncols`
+// and keeps every listed row aligned for its vector loads.
 int pick_nc(int ncols, int elem, const void* p0, int64_t ld0, const void* p1, int64_t ld1) {
-  int nc = 16 / elem;
-  while (nc > 1 && !((ncols % nc) == 0 && aligned(p0, ld0, nc, elem) && aligned(p1, ld1, nc, elem))) nc >>= 1;
+  int nc = 32 / elem;
+  auto ok = [&](int c) {
+    const int vec = std::min(c, 16 / elem);  // elements per vector access
+    return (ncols % c) == 0 && aligned(p0, ld0, vec, elem) && aligned(p1, ld1, vec, elem);
+  };
+  while (nc > 1 && !ok(nc)) nc >>= 1;
   return nc;
 }
 
@@ -586,18 +613,18 @@ cudaError_t launch_pdl(void (*kern)(const Args), dim3 grid, cudaStream_t s, cons
 template <typename T, bool TRANS>
 using SpmmKernel = void (*)(const SpmmArgs<T>);
 
-// Instantiated shapes: NC = 16 bytes' worth of elements with G = 1..8 (bf16) / 1..16
-// (fp32) lanes, narrower vectors with one lane, and scalars with G = 1..32.
+// Instantiated shapes: 32-byte groups (NC = 16 bf16 / 8 fp32) with G = 1..64/NC lanes,
+// 16-, 8- and 4-byte groups with one lane, and scalars with G = 1..32.
 template <typename T, bool TRANS>
 SpmmKernel<T, TRANS> pick_spmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
   if (nc == NC_ && g == G_) return k_spmm_small<T, NC_, G_, TRANS>;
   if constexpr (sizeof(T) == 2) {
+    SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4)
+    SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
+  } else {
     SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(8, 4) SNK_CASE(8, 8)
     SNK_CASE(4, 1) SNK_CASE(2, 1)
-  } else {
-    SNK_CASE(4, 1) SNK_CASE(4, 2) SNK_CASE(4, 4) SNK_CASE(4, 8) SNK_CASE(4, 16)
-    SNK_CASE(2, 1)
   }
   SNK_CASE(1, 1) SNK_CASE(1, 2) SNK_CASE(1, 4) SNK_CASE(1, 8) SNK_CASE(1, 16) SNK_CASE(1, 32)
 #undef SNK_CASE
@@ -612,11 +639,11 @@ SddmmKernel<T> pick_sddmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
   if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_>;
   if constexpr (sizeof(T) == 2) {
+    SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4) SNK_CASE(16, 8) SNK_CASE(16, 16) SNK_CASE(16, 32)
+    SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
+  } else {
     SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(8, 4) SNK_CASE(8, 8) SNK_CASE(8, 16) SNK_CASE(8, 32)
     SNK_CASE(4, 1) SNK_CASE(2, 1)
-  } else {
-    SNK_CASE(4, 1) SNK_CASE(4, 2) SNK_CASE(4, 4) SNK_CASE(4, 8) SNK_CASE(4, 16) SNK_CASE(4, 32)
-    SNK_CASE(2, 1)
   }
   SNK_CASE(1, 1) SNK_CASE(1, 2) SNK_CASE(1, 4) SNK_CASE(1, 8) SNK_CASE(1, 16) SNK_CASE(1, 32)
 #undef SNK_CASE
@@ -634,7 +661,7 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     T* Cc = C + col0;
     int nc = pick_nc(ncols, elem, Bc, ldb, Cc, ldc);
     int g = pow2ceil((ncols + nc - 1) / nc);
-    const int gmax = nc == 1 ? 32 : (elem == 2 ? (nc == 8 ? 8 : 1) : (nc == 4 ? 16 : 1));
+    const int gmax = nc == 1 ? 32 : (nc * elem == 32 ? 64 / nc : 1);
     if (g > gmax) {  // narrow vectors come with one lane only: use scalars instead
       nc = 1;
       g = pow2ceil(ncols);
@@ -658,6 +685,7 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     A.nnz = L->nnz;
     A.P = L->P;
     A.ncols = ncols;
+    A.b32 = (TRANS ? L->M : L->K) * ldb <= (int64_t)0xffffffffLL ? 1 : 0;
     A.carry_tail = TRANS ? L->carry_tail_b : L->carry_tail_f;
     A.carry_head = TRANS ? L->carry_head_b : L->carry_head_f;
     A.cnt = TRANS ? L->cnt_b : L->cnt_f;
