@@ -92,13 +92,21 @@ def barrier(world: int):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_per_step_max: float) -> float:
+    """Whole-job rate: every rank processes units_per_rank per step (weak scaling, replicas),
+    and the step time is the maximum over ranks."""
+    return units_per_rank * world / (ms_per_step_max * 1e-3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -192,12 +200,14 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
     # build R copies (timing the build of the first)
     copies = []
     t_build = None
+    ws_bytes = snk.snk_workspace_bytes(M, K, nnz, args.parts)
     for i in range(R):
         row, col, val = torch.from_numpy(row_h).to(dev), torch.from_numpy(col_h).to(dev), dev_bf16(val_h)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            t0 = time.perf_counter()
-            L = snk.Layout(M, K, row, col, val, num_parts=args.parts)
+            t0 = time.perf_counter()  # the build call alone (it ends with its own stream sync)
+            L = snk.Layout(M, K, row, col, val, num_parts=args.parts, workspace=ws)
             t1 = time.perf_counter()
         if i == 0:
             t_build = t1 - t0
@@ -290,8 +300,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
 
     step_bytes = sum(op_bytes(op, M, K, nnz, N, s) for N in batches for op in OPS)
     step_flops = sum(op_flops(nnz, N) for N in batches for op in OPS)
-    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
-    gflops = step_flops * world / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, ms_per_step) / 1e9
+    gflops = job_throughput(step_flops, world, ms_per_step) / 1e9
 
     # end to end through the public API: pinned host inputs in, results out, every step
     pinned = {}
@@ -329,7 +339,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
     e1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    e2e_value = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+    e2e_value = job_throughput(step_bytes, world, e2e_ms) / 1e9
 
     # preprocessing: build (timed above, host wall clock incl. its one sync) and one restructure
     L0 = copies[0]["L"]
@@ -481,6 +491,39 @@ def run_reference(args, rank: int, world: int) -> dict:
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile(args) -> None:
+    """Two passes of the step's launches on one layout, no timing: pass 0 warms up, pass 1 is
+    what an ncu capture selects (-s 3*len(batches) -c 3*len(batches)).  For profiling only."""
+    import torch
+
+    from sparse_spmm_b200 import build as build_mod
+    from sparse_spmm_b200 import snk
+    from sparse_spmm_b200 import workloads as wl
+
+    build_mod.build()
+    torch.cuda.set_device(0)
+    layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
+
+    def dev_t(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(a).cuda()
+
+    L = snk.Layout(layer.M, layer.K, dev_t(layer.row), dev_t(layer.col), dev_t(layer.values), num_parts=args.parts)
+    batches = [int(b) for b in args.batches.split(",")]
+    data = {N: (dev_t(wl.activations(layer.K, N, "bf16", args.seed, stream=2)),
+                dev_t(wl.activations(layer.M, N, "bf16", args.seed, stream=3))) for N in batches}
+    torch.cuda.synchronize()
+    for _ in range(2):
+        for N in batches:
+            X, dY = data[N]
+            L.forward(X)
+            L.backward_input(dY)
+            L.backward_weight(dY, X)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_passes": 2, "launches_per_pass": 3 * len(batches), "batches": batches}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -493,10 +536,15 @@ def main():
     ap.add_argument("--rotate", type=int, default=0, help="number of rotated copies (0 = enough for 3x L2)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run two untimed passes of the step (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.profile:
+        run_profile(args)
+        return 0
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))

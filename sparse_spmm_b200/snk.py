@@ -189,7 +189,7 @@ class Layout:
     """
 
     def __init__(self, M: int, K: int, row: torch.Tensor, col: torch.Tensor, values: torch.Tensor,
-                 num_parts: int = 0, stream=None):
+                 num_parts: int = 0, stream=None, workspace: torch.Tensor | None = None):
         if row.dtype != torch.int32 or col.dtype != torch.int32:
             raise TypeError("row/col must be int32")
         if not (row.is_cuda and col.is_cuda and values.is_cuda):
@@ -202,7 +202,11 @@ class Layout:
         nbytes = snk_workspace_bytes(self.M, self.K, row.numel(), num_parts)
         if nbytes == 0:
             raise SnkError(1, "snk_workspace_bytes")
-        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=row.device)
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=row.device)
+        elif workspace.dtype != torch.uint8 or workspace.numel() < nbytes or not workspace.is_contiguous():
+            raise ValueError(f"workspace must be a contiguous uint8 tensor of >= {nbytes} bytes")
+        self.workspace = workspace
         self.handle = snk_build(self.M, self.K, row, col, values, num_parts, self.workspace, stream)
         info = snk_layout_info(self.handle)
         self.nnz = int(info.nnz)

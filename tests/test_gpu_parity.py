@@ -116,7 +116,7 @@ def test_conv1x1_sweep_sampled(shape, sparsity):
 # ----------------------------------------------------------------------------- edge cases
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("N", [1, 2, 3, 5, 31, 33, 64, 65, 130])
+@pytest.mark.parametrize("N", [1, 2, 3, 5, 31, 33, 64, 65, 72, 130, 264])
 def test_ragged_batches(dtype, N):
     layer = wl.uniform_layer(300, 211, 0.93, dtype, 3, "W")
     L = gpu_layout(layer)
@@ -130,7 +130,7 @@ def test_padded_leading_dimension(pad):
         layer = wl.uniform_layer(257, 190, 0.9, dtype, 5, "W")
         L = gpu_layout(layer)
         ref = check_build(L, layer)
-        for N in (1, 8, 17, 32):
+        for N in (1, 8, 17, 32, 96):
             check_products(layer, ref, L, N, seed=7, pad=pad)
 
 
@@ -149,7 +149,7 @@ def test_partition_counts(P):
         L = gpu_layout(layer, num_parts=P)
         assert L.num_parts == min(P, layer.nnz)
         ref = check_build(L, layer)
-        for N in (1, 8, 40):
+        for N in (1, 8, 40, 136):
             check_products(layer, ref, L, N, seed=N)
 
 
@@ -176,6 +176,21 @@ def test_empty_and_degenerate_shapes():
     L = gpu_layout(layer)
     ref = check_build(L, layer)
     check_products(layer, ref, L, 4)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [2048, 2056])
+def test_wide_batches(dtype, N):
+    # the row-block x column-slice kernel: several slices, a ragged last slice, long rows
+    rng = np.random.default_rng(N)
+    M, K = 150, 700
+    lin = set(rng.choice(M * K, size=9000, replace=False).tolist()) | {33 * K + c for c in range(K)}
+    lin = np.array(sorted(lin))
+    lin = lin[rng.permutation(lin.size)]
+    layer = explicit_layer(M, K, lin // K, lin % K, rng.normal(0, 0.02, size=lin.size).astype(np.float32), dtype)
+    L = gpu_layout(layer)
+    ref = check_build(L, layer)
+    check_products(layer, ref, L, N, seed=3, ops=("forward", "backward_input"))
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
