@@ -61,8 +61,17 @@ struct Packed {
 };
 
 template <int NC, typename T>
-__device__ __forceinline__ void load_packed(const T* p, Packed<T, NC>& r) {
+__device__ __forceinline__ void load_packed(const T* p, Packed<T, NC>& r, bool a32 = false) {
   constexpr int W = Packed<T, NC>::W;
+  if constexpr (W == 8) {
+    if (a32) {  // one 32-byte load
+      asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                   : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]),
+                     "=r"(r.w[6]), "=r"(r.w[7])
+                   : "l"(p));
+      return;
+    }
+  }
   if constexpr (W >= 4) {
 #pragma unroll
     for (int k = 0; k < W; k += 4) {
@@ -96,20 +105,28 @@ __device__ __forceinline__ float unpack(const Packed<T, NC>& r, int j) {
   }
 }
 
+// NC fp32 accumulators held as register pairs, so packed FMAs need no repacking.
+template <int NC>
+struct Acc {
+  float2 p[(NC + 1) / 2];
+  __device__ __forceinline__ float& operator[](int j) { return (j & 1) ? p[j >> 1].y : p[j >> 1].x; }
+  __device__ __forceinline__ float operator[](int j) const { return (j & 1) ? p[j >> 1].y : p[j >> 1].x; }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int k = 0; k < (NC + 1) / 2; ++k) p[k] = make_float2(0.f, 0.f);
+  }
+};
+
 // acc[j] += v * x[j] for the NC columns, two columns per packed fp32 FMA.
 template <typename T, int NC>
-__device__ __forceinline__ void fma_row(float v, const Packed<T, NC>& x, float* acc) {
+__device__ __forceinline__ void fma_row(float v, const Packed<T, NC>& x, Acc<NC>& acc) {
   if constexpr (NC == 1) {
-    acc[0] = fmaf(v, unpack<T, NC>(x, 0), acc[0]);
+    acc.p[0].x = fmaf(v, unpack<T, NC>(x, 0), acc.p[0].x);
   } else {
     const float2 vv = make_float2(v, v);
 #pragma unroll
-    for (int j = 0; j < NC; j += 2) {
-      float2 a2 = make_float2(acc[j], acc[j + 1]);
-      a2 = __ffma2_rn(vv, make_float2(unpack<T, NC>(x, j), unpack<T, NC>(x, j + 1)), a2);
-      acc[j] = a2.x;
-      acc[j + 1] = a2.y;
-    }
+    for (int j = 0; j < NC; j += 2)
+      acc.p[j / 2] = __ffma2_rn(vv, make_float2(unpack<T, NC>(x, j), unpack<T, NC>(x, j + 1)), acc.p[j / 2]);
   }
 }
 
@@ -145,6 +162,14 @@ __device__ __forceinline__ void store_cols(T* p, const float* v) {
       p[0] = v[0];
     }
   }
+}
+
+template <int NC, typename T>
+__device__ __forceinline__ void store_cols(T* p, const Acc<NC>& a) {
+  float v[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) v[j] = a[j];
+  store_cols<NC>(p, v);
 }
 
 template <int NC, typename T>
@@ -199,6 +224,7 @@ struct SpmmArgs {
   int P;
   int ncols;           // columns in this launch (<= kCarryCols, a multiple of NC)
   int b32;             // every gathered row offset c * ldb fits in 32 bits
+  int a32;             // every gathered lane group is 32-byte aligned
   float* carry_tail;   // [P][kCarryCols]
   float* carry_head;   // [P][kCarryCols]
   uint32_t* cnt;       // [kMaxTiles][P], zero between launches
@@ -269,10 +295,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   T* __restrict__ Cb = A.C + n0;
   const unsigned ldb = (unsigned)A.ldb;
   const bool small_b = A.b32 != 0;
+  const bool a32 = A.a32 != 0;
 
-  float acc[NC];
-#pragma unroll
-  for (int j = 0; j < NC; ++j) acc[j] = 0.f;
+  Acc<NC> acc;
+  acc.zero();
   bool has_head = false, has_tail = false, link = true;
   int64_t h_row = -1;
 
@@ -294,8 +320,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
       }
       first = false;
       open = false;
-#pragma unroll
-      for (int j = 0; j < NC; ++j) acc[j] = 0.f;
+      acc.zero();
     };
 
     int e = s;
@@ -308,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
         vv[i] = v[i];
         if (i < nb && active) {
           const T* src = small_b ? Bb + (unsigned)c[i] * ldb : Bb + (int64_t)c[i] * A.ldb;
-          load_packed<NC>(src, x[i]);
+          load_packed<NC>(src, x[i], a32);
         } else {
           zero_packed(x[i]);
         }
@@ -431,7 +456,12 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   }
   if (w == NW - 1 && np > 0) {
     const int64_t t = search_row([&](int64_t q) { return (int64_t)RP(q); }, ra, mn64(rb, A.rows - 1), np - 1);
-    if (RP(t + 1) > np) cross_cta(t, acc, false);
+    if (RP(t + 1) > np) {
+      float tv[NC];
+#pragma unroll
+      for (int j = 0; j < NC; ++j) tv[j] = acc[j];
+      cross_cta(t, tv, false);
+    }
   }
 }
 
@@ -449,6 +479,7 @@ struct SddmmArgs {
   int64_t rows;
   int64_t nnz;
   int N;             // a multiple of NC
+  int a32;           // X and dY lane groups are 32-byte aligned
 };
 
 template <typename T, int NC>
@@ -495,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
       if (i < nb) c[i] = __ldg(col + e0 + i);
   };
   if (s < e_end) load_batch(s, min(UB, e_end - s));
+  const bool a32 = A.a32 != 0;
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
   const bool in_smem = np > 0 && span <= kRowCap;
@@ -532,10 +564,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
         Packed<T, NC> xv[UB];
 #pragma unroll
         for (int i = 0; i < UB; ++i)
-          if (i < nb) load_packed<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, xv[i]);
+          if (i < nb) load_packed<NC>(A.X + (int64_t)cc[i] * A.ldx + n0, xv[i], a32);
         if (one_row) {
           Packed<T, NC> yv;
-          load_packed<NC>(A.dY + (int64_t)rr[0] * A.lddy + n0, yv);
+          load_packed<NC>(A.dY + (int64_t)rr[0] * A.lddy + n0, yv, a32);
 #pragma unroll
           for (int i = 0; i < UB; ++i)
             if (i < nb) d[i] = dot_packed(xv[i], yv, d[i]);
@@ -544,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
           for (int i = 0; i < UB; ++i) {
             if (i < nb) {
               Packed<T, NC> yv;
-              load_packed<NC>(A.dY + (int64_t)rr[i] * A.lddy + n0, yv);
+              load_packed<NC>(A.dY + (int64_t)rr[i] * A.lddy + n0, yv, a32);
               d[i] = dot_packed(xv[i], yv, d[i]);
             }
           }
@@ -953,6 +985,7 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     A.P = L->P;
     A.ncols = ncols;
     A.b32 = (TRANS ? L->M : L->K) * ldb <= (int64_t)0xffffffffLL ? 1 : 0;
+    A.a32 = (nc * elem == 32 && ((uintptr_t)Bc % 32) == 0 && ((ldb * elem) % 32) == 0) ? 1 : 0;
     A.carry_tail = TRANS ? L->carry_tail_b : L->carry_tail_f;
     A.carry_head = TRANS ? L->carry_head_b : L->carry_head_f;
     A.cnt = TRANS ? L->cnt_b : L->cnt_f;
@@ -987,6 +1020,8 @@ snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* 
   A.rows = L->M;
   A.nnz = L->nnz;
   A.N = (int)N;
+  A.a32 = (nc * elem == 32 && ((uintptr_t)X % 32) == 0 && ((uintptr_t)dY % 32) == 0 && ((ldx * elem) % 32) == 0 &&
+           ((lddy * elem) % 32) == 0) ? 1 : 0;
   SNK_CUDA_TRY(launch_pdl(kern, dim3((unsigned)L->P), s, A));
   return SNK_OK;
 }
