@@ -188,6 +188,22 @@ __device__ __forceinline__ void store_zero(T* p) {
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Bulk L2 prefetch of the 16-byte-aligned bytes inside [p, p + bytes).  Only a hint: L2 is
+// the point of coherence, so it may run before the previous grid has finished writing.
+__device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes) {
+  const uintptr_t lo = ((uintptr_t)p + 15) & ~(uintptr_t)15;
+  const uintptr_t hi = ((uintptr_t)p + (uintptr_t)bytes) & ~(uintptr_t)15;
+  if (bytes > 0 && hi > lo && hi - lo < (1u << 30))
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo), "r"((uint32_t)(hi - lo)) : "memory");
+}
+
+// Slice part of P of an array of n elements of E bytes: [n * part / P, n * (part + 1) / P).
+template <int E>
+__device__ __forceinline__ void prefetch_slice(const void* base, int64_t n, int part, int P) {
+  const int64_t i0 = n * part / P, i1 = n * (part + 1) / P;
+  prefetch_l2(static_cast<const char*>(base) + i0 * E, (i1 - i0) * E);
+}
+
 // f(integral_constant<int, I>) for I = B .. E-1, unrolled at compile time.
 template <int B, int E, typename F>
 __device__ __forceinline__ void static_for(F&& f) {
@@ -225,14 +241,22 @@ struct SpmmArgs {
   int ncols;           // columns in this launch (<= kCarryCols, a multiple of NC)
   int b32;             // every gathered row offset c * ldb fits in 32 bits
   int a32;             // every gathered lane group is 32-byte aligned
+  int64_t bbytes;      // bytes of the gathered operand when it is one dense block, else 0
+  int64_t prows;       // entries of ptr
   float* carry_tail;   // [P][kCarryCols]
   float* carry_head;   // [P][kCarryCols]
   uint32_t* cnt;       // [kMaxTiles][P], zero between launches
 };
 
+// Transposed, with 16- or 32-byte lane groups, the value positions are loaded one batch ahead
+// of the values (the batches are long enough for the second stage to pay).
+template <typename T, int NC, bool TRANS>
+constexpr bool perm_ahead() { return TRANS && NC * (int)sizeof(T) >= 16; }
 // Entries in flight per worker: as many as the register budget of 3 CTAs per SM allows.
-template <typename T, int NC>
-constexpr int spmm_batch() { return NC * (int)sizeof(T) >= 32 ? 3 : (NC * (int)sizeof(T) >= 16 ? 6 : 8); }
+template <typename T, int NC, bool TRANS = false>
+constexpr int spmm_batch() {
+  return NC * (int)sizeof(T) >= 32 ? 3 : (NC * (int)sizeof(T) >= 16 ? (perm_ahead<T, NC, TRANS>() ? 5 : 6) : 8);
+}
 template <typename T, int NC>
 constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 32 ? 2 : (NC * (int)sizeof(T) >= 8 ? 4 : 6); }
 
@@ -242,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   constexpr int WPW = 32 / G;        // workers per warp
   constexpr int NT = NC * G;         // columns per tile
   constexpr int NWARPS = kThreads / 32;
-  constexpr int UB = spmm_batch<T, NC>();
+  constexpr int UB = spmm_batch<T, NC, TRANS>();
+  constexpr bool PA = perm_ahead<T, NC, TRANS>();
   __shared__ int32_t s_rp[kRowCap];
   __shared__ float s_agg[NWARPS][NT];
   __shared__ int s_aggF[NWARPS];
@@ -256,6 +281,21 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
   const int n0 = tile * NT + l * NC;
   const bool active = n0 < A.ncols;  // this lane holds NC real columns (or none)
+  if (tile == 0 && lane == 0) {
+    // L2 warm-up while the previous grid drains: together the CTAs cover every operand once.
+    if (wp == 0) {
+      prefetch_l2(A.desc + part, sizeof(int4));
+      prefetch_slice<4>(A.ptr, A.prows, part, A.P);
+    } else if (wp == 1) {
+      prefetch_slice<4>(A.idx, A.nnz, part, A.P);
+    } else if (wp == 2) {
+      prefetch_slice<sizeof(T)>(A.vals, A.nnz, part, A.P);
+    } else if (wp == 3) {
+      if (TRANS) prefetch_slice<4>(A.perm, A.nnz, part, A.P);
+    } else if (wp == 4) {
+      prefetch_slice<1>(A.B, A.bbytes, part, A.P);
+    }
+  }
   pdl_wait();
 
   const int4 dsc = __ldg(A.desc + part);
@@ -268,19 +308,34 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   const int32_t* __restrict__ prm = TRANS ? A.perm + a : nullptr;
   const T* __restrict__ vals = TRANS ? A.vals : A.vals + a;
 
-  // the worker's next batch of indices / values (prefetched one batch ahead)
+  // the worker's next batch of indices / values (prefetched one batch ahead); with PA the
+  // value positions run one batch further ahead, so each value gather waits on one load only
   int c[UB];
   float v[UB];
+  int pn[PA ? UB : 1];
+  auto load_perm = [&](int e0, int nb) {
+    if constexpr (PA) {
+#pragma unroll
+      for (int i = 0; i < UB; ++i)
+        if (i < nb) pn[i] = __ldg(prm + e0 + i);
+    }
+  };
   auto load_batch = [&](int e0, int nb) {
 #pragma unroll
     for (int i = 0; i < UB; ++i) {
       if (i < nb) {
         c[i] = __ldg(idx + e0 + i);
-        v[i] = TRANS ? load1(vals + __ldg(prm + e0 + i)) : load1(vals + e0 + i);
+        if constexpr (PA) v[i] = load1(vals + pn[i]);
+        else v[i] = TRANS ? load1(vals + __ldg(prm + e0 + i)) : load1(vals + e0 + i);
       }
     }
+    const int e1 = e0 + nb;  // the batch after this one
+    if (PA && e1 < e_end) load_perm(e1, min(UB, e_end - e1));
   };
-  if (s < e_end) load_batch(s, min(UB, e_end - s));
+  if (s < e_end) {
+    load_perm(s, min(UB, e_end - s));
+    load_batch(s, min(UB, e_end - s));
+  }
 
   const int64_t rhi = mn64(rb + 1, A.rows);
   const int64_t span = rhi - ra + 1;
@@ -480,6 +535,7 @@ struct SddmmArgs {
   int64_t nnz;
   int N;             // a multiple of NC
   int a32;           // X and dY lane groups are 32-byte aligned
+  int64_t xbytes, dybytes;  // bytes of X and dY when each is one dense block, else 0
 };
 
 template <typename T, int NC>
@@ -510,6 +566,20 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
   const int w = tid / G, l = tid % G;
   const int lane_base = lane - l;
   const unsigned gmask = G == 32 ? kFull : (((1u << G) - 1u) << lane_base);
+  if (lane == 0) {
+    // L2 warm-up while the previous grid drains: together the CTAs cover every operand once.
+    const int wp = tid >> 5, P = (int)gridDim.x;
+    if (wp == 0) {
+      prefetch_l2(A.desc + part, sizeof(int4));
+      prefetch_slice<4>(A.row_ptr, A.rows + 1, part, P);
+    } else if (wp == 1) {
+      prefetch_slice<4>(A.col, A.nnz, part, P);
+    } else if (wp == 2) {
+      prefetch_slice<1>(A.X, A.xbytes, part, P);
+    } else if (wp == 3) {
+      prefetch_slice<1>(A.dY, A.dybytes, part, P);
+    }
+  }
   pdl_wait();
 
   const int4 dsc = __ldg(A.desc + part);
@@ -986,6 +1056,8 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     A.ncols = ncols;
     A.b32 = (TRANS ? L->M : L->K) * ldb <= (int64_t)0xffffffffLL ? 1 : 0;
     A.a32 = (nc * elem == 32 && ((uintptr_t)Bc % 32) == 0 && ((ldb * elem) % 32) == 0) ? 1 : 0;
+    A.bbytes = (ldb == ncols) ? (TRANS ? L->M : L->K) * ldb * elem : 0;
+    A.prows = rows + 1;
     A.carry_tail = TRANS ? L->carry_tail_b : L->carry_tail_f;
     A.carry_head = TRANS ? L->carry_head_b : L->carry_head_f;
     A.cnt = TRANS ? L->cnt_b : L->cnt_f;
@@ -1022,6 +1094,8 @@ snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* 
   A.N = (int)N;
   A.a32 = (nc * elem == 32 && ((uintptr_t)X % 32) == 0 && ((uintptr_t)dY % 32) == 0 && ((ldx * elem) % 32) == 0 &&
            ((lddy * elem) % 32) == 0) ? 1 : 0;
+  A.xbytes = ldx == N ? L->K * N * elem : 0;
+  A.dybytes = lddy == N ? L->M * N * elem : 0;
   SNK_CUDA_TRY(launch_pdl(kern, dim3((unsigned)L->P), s, A));
   return SNK_OK;
 }
