@@ -524,6 +524,159 @@ def run_profile(args) -> None:
     print(json.dumps({"profile_passes": 2, "launches_per_pass": 3 * len(batches), "batches": batches}))
 
 
+# ----------------------------------------------------------------------------- sweep over every config
+
+def _graph_time_us(fns, reps: int = 3, rounds: int = 3) -> float:
+    """Per-call µs of the calls in `fns` (one per rotated copy), captured into one CUDA graph
+    and replayed `reps` times; best of `rounds`."""
+    import torch
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):  # eager warm-up: library handles (cuBLAS) exist before capture
+        for f in fns:
+            f()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for f in fns:
+            f()
+    with torch.cuda.stream(s):
+        g.replay()
+    s.synchronize()
+    best = float("inf")
+    for _ in range(rounds):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                g.replay()
+            e1.record(s)
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e3 / (reps * len(fns)))
+    del g
+    return best
+
+
+def fp32_fma_peak(sm_count: int) -> dict:
+    """Measured fp32 FMA rate (TFLOP/s) from the library's probe, best of 3 ~10 ms launches."""
+    import torch
+    from sparse_spmm_b200 import snk
+    blocks = 4 * sm_count
+    sink = torch.zeros(blocks, device="cuda")
+    iters = 60000
+    snk.snk_probe_fp32_fma(blocks, 1000, sink)
+    best = float("inf")
+    flops = 0
+    for _ in range(3):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        flops = snk.snk_probe_fp32_fma(blocks, iters, sink)
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e-3)
+    return {"tflops": round(flops / best / 1e12, 2), "blocks": blocks, "iters": iters}
+
+
+def run_sweep(args) -> None:
+    """Every config, op and batch of the workload list: L2-cold per-op CUDA graphs, achieved
+    GB/s and GFLOP/s under the byte model, fractions of the measured HBM and fp32 FMA peaks,
+    and (forward) the dense and dense+mask products of the same W on the same GPU
+    (torch.matmul, i.e. cuBLAS), as the pages' ratio style.  One JSON line per measurement."""
+    import torch
+
+    from sparse_spmm_b200 import build as build_mod
+    from sparse_spmm_b200 import snk
+    from sparse_spmm_b200 import workloads as wl
+
+    build_mod.build()
+    torch.cuda.set_device(0)
+    sm_count = torch.cuda.get_device_properties(0).multi_processor_count
+    pk = peaks()
+    l2 = 126 * 2 ** 20
+
+    def dev_t(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    with ClockSampler(0) as clk:
+        f32 = fp32_fma_peak(sm_count)
+    f32["clocks"] = clk.summary()
+    print(json.dumps({"sweep": "fp32_fma_peak", **f32}), flush=True)
+
+    works = [wl.tiny_fc(), wl.fc_4096(), wl.gpt2_mlp(), wl.llama_mlp()]
+    works += [wl.conv1x1(M, K, sp) for (M, K) in wl.CONV_SHAPES for sp in wl.CONV_SPARSITIES]
+    opname = {"forward": "forward", "backward_input": "backward_input", "backward_weight": "backward_weight"}
+    for work in works:
+        s = 2 if work.dtype == "bf16" else 4
+        tdt = torch.bfloat16 if work.dtype == "bf16" else torch.float32
+        for make in work.layers:
+            layer = make()
+            M, K, nnz = layer.M, layer.K, layer.nnz
+            hot = nnz * (s + 12) + 8 * (M + K) + max(work.batches) * (M + K) * s * 2
+            R = int(min(40, max(2, np.ceil(3 * l2 / hot))))
+            copies = [snk.Layout(M, K, dev_t(layer.row), dev_t(layer.col), dev_t(layer.values)) for _ in range(R)]
+            for N in work.batches:
+                X = [dev_t(wl.activations(K, N, work.dtype, args.seed, 2, work.relu_x)) for _ in range(R)]
+                dY = [dev_t(wl.activations(M, N, work.dtype, args.seed, 3)) for _ in range(R)]
+                Y = [torch.empty(M, N, dtype=tdt, device="cuda") for _ in range(R)]
+                dX = [torch.empty(K, N, dtype=tdt, device="cuda") for _ in range(R)]
+                dW = [torch.empty(nnz, dtype=tdt, device="cuda") for _ in range(R)]
+                torch.cuda.synchronize()
+                for op in work.ops:
+                    if op == "restructure":
+                        continue
+                    if op == "forward":
+                        fns = [lambda i=i: copies[i].forward(X[i], Y=Y[i]) for i in range(R)]
+                    elif op == "backward_input":
+                        fns = [lambda i=i: copies[i].backward_input(dY[i], dX=dX[i]) for i in range(R)]
+                    else:
+                        fns = [lambda i=i: copies[i].backward_weight(dY[i], X[i], dW=dW[i]) for i in range(R)]
+                    us = _graph_time_us(fns, reps=3 if N >= 1024 else 10)
+                    b = op_bytes(opname[op], M, K, nnz, N, s)
+                    fl = op_flops(nnz, N)
+                    rec = {"sweep": work.name, "layer": layer.name, "M": M, "K": K, "nnz": nnz, "op": op, "N": N,
+                           "us": round(us, 2), "gbs": round(b / us / 1e3, 1),
+                           "frac_hbm": round(b / us / 1e3 / pk["hbm_gbs"], 4),
+                           "gflops": round(fl / us / 1e3, 1), "frac_fp32": round(fl / us / 1e6 / f32["tflops"], 4),
+                           "bound": "alu" if fl / (f32["tflops"] * 1e12) > b / (pk["hbm_gbs"] * 1e9) else "hbm"}
+                    if op == "forward":
+                        # dense and dense+mask products of the same W (cuBLAS via torch), L2-cold too
+                        Wd = torch.zeros(M, K, dtype=tdt, device="cuda")
+                        Wd[dev_t(layer.row).long(), dev_t(layer.col).long()] = dev_t(layer.values)
+                        Md = (Wd != 0).to(tdt)
+                        Rd = int(min(R, max(2, np.ceil(3 * l2 / (M * K * s * 2 + (M + K) * N * s)))))
+                        Wds = [Wd.clone() for _ in range(Rd)]
+                        Mds = [Md.clone() for _ in range(Rd)]
+                        Tmp = [torch.empty_like(Wd) for _ in range(Rd)]
+                        dense = [lambda i=i: torch.matmul(Wds[i], X[i], out=Y[i]) for i in range(Rd)]
+                        masked = [lambda i=i: (torch.mul(Wds[i], Mds[i], out=Tmp[i]),
+                                               torch.matmul(Tmp[i], X[i], out=Y[i])) for i in range(Rd)]
+                        rec["dense_us"] = round(_graph_time_us(dense), 2)
+                        rec["dense_mask_us"] = round(_graph_time_us(masked), 2)
+                        rec["speedup_vs_dense"] = round(rec["dense_us"] / us, 2)
+                        rec["speedup_vs_dense_mask"] = round(rec["dense_mask_us"] / us, 2)
+                        del Wd, Md, Wds, Mds, Tmp
+                    print(json.dumps(rec), flush=True)
+                del X, dY, Y, dX, dW
+            if "restructure" in work.ops:
+                k = int(round(0.1 * nnz))
+                L = copies[0]
+                L.restructure(k, seed=args.seed)  # warm-up
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                L.restructure(k, seed=args.seed + 1)
+                e1.record()
+                e1.synchronize()
+                print(json.dumps({"sweep": work.name, "layer": layer.name, "op": "restructure", "drop": k,
+                                  "ms": round(e0.elapsed_time(e1), 3)}), flush=True)
+            del copies
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -538,12 +691,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run two untimed passes of the step (for ncu captures) and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every config, op and batch (plus dense baselines); JSON lines; exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     if args.profile:
         run_profile(args)
+        return 0
+    if args.sweep:
+        run_sweep(args)
         return 0
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

@@ -190,6 +190,27 @@ SNK_API snk_status snk_csr_forward_static(int64_t M, int64_t K, int64_t nnz, con
 
 /* Fill *v with the layout's sizes and device pointers.  Returns SNK_ERR_INVALID_ARG for
  * NULL arguments. */
+/*
+ * snk_sync_status -- synchronises `stream` and reports whether a product launch on this
+ * layout gave up a bounded wait: the TMA-staged kernels for wide operands wait on
+ * shared-memory barriers for the tensor copies, each wait for at most about a second.
+ * Returns SNK_ERR_TIMEOUT then (and clears the layout's status word), SNK_OK otherwise.
+ * The products never synchronise; this is how a caller that wants to know checks.
+ * (A library addition; the paper has no counterpart.)
+ */
+SNK_API snk_status snk_sync_status(snk_layout* L, snk_stream stream);
+
+/*
+ * snk_probe_fp32_fma -- a measurement aid, not part of the method: launches `blocks` CTAs
+ * of chains of packed fp32 FMAs, `iters` steps each, on `stream`, so that a caller timing
+ * it with events learns the GPU's fp32 FMA rate (the ALU roofline of the products when
+ * N is large).  snk_probe_fp32_fma_flops returns the floating-point operations of such a
+ * launch (an FMA counts 2).  sink: device float [blocks], normally left unwritten.
+ * Asynchronous; SNK_ERR_INVALID_ARG for blocks or iters <= 0 or a NULL sink.
+ */
+SNK_API snk_status snk_probe_fp32_fma(int32_t blocks, int32_t iters, float* sink, snk_stream stream);
+SNK_API int64_t snk_probe_fp32_fma_flops(int32_t blocks, int32_t iters);
+
 SNK_API snk_status snk_layout_info(const snk_layout* L, snk_layout_view* v);
 
 /* Free the host object (no device memory is freed; the caller owns the workspace). */

@@ -14,6 +14,7 @@ enum : uint32_t {
   ERRBIT_OUT_OF_RANGE = 1u,
   ERRBIT_DUPLICATE = 2u,
   ERRBIT_INVALID_VALUE = 4u,
+  ERRBIT_TIMEOUT = 8u,  // a bounded wait of a product kernel gave up
 };
 
 // Columns covered by one launch of the small-N SpMM kernels; the cross-CTA carry slots

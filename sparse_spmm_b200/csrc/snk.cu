@@ -180,6 +180,20 @@ snk_status snk_restructure(snk_layout* L, void* values, int64_t drop_count, uint
   });
 }
 
+snk_status snk_sync_status(snk_layout* L, snk_stream stream) {
+  if (L == nullptr) return SNK_ERR_INVALID_ARG;
+  return on_device(L->device, [&]() -> snk_status {
+    const cudaStream_t s = (cudaStream_t)stream;
+    uint32_t e = 0;
+    SNK_CUDA_TRY(cudaMemcpyAsync(&e, L->err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
+    SNK_CUDA_TRY(cudaStreamSynchronize(s));
+    if ((e & snk::ERRBIT_TIMEOUT) == 0) return SNK_OK;
+    SNK_CUDA_TRY(cudaMemsetAsync(L->err, 0, sizeof(uint32_t), s));
+    SNK_CUDA_TRY(cudaStreamSynchronize(s));
+    return SNK_ERR_TIMEOUT;
+  });
+}
+
 snk_status snk_layout_info(const snk_layout* L, snk_layout_view* v) {
   if (L == nullptr || v == nullptr) return SNK_ERR_INVALID_ARG;
   v->M = L->M;

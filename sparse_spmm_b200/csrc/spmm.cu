@@ -27,6 +27,11 @@
 #include <algorithm>
 #include <type_traits>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace snk {
@@ -704,6 +709,7 @@ struct WideArgs {
   int64_t rows, brows;
   int N;
   int rb;               // rows per CTA (8 * rows per warp, <= 8 * kWideRW)
+  uint32_t* err;        // status word (may be null): ERRBIT_TIMEOUT if a pipeline wait gave up
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
@@ -875,12 +881,237 @@ __global__ void __launch_bounds__(kThreads, 2) k_spmm_wide(const WideArgs<T> A) 
     const int64_t r = r0 + wp * rw + i;
     if (i < rw && r < A.rows && c0 < ncols) {
       T* dst = A.C + r * A.ldc + n0 + c0;
-      if (c0 + 4 <= ncols) {
+      if (c0 + 4 <= ncols && ((uintptr_t)dst % (4 * E)) == 0) {  // one vector store where aligned
         store_cols<4>(dst, acc[i]);
       } else {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (j < ncols - c0) store1(dst + j, acc[i][j]);
+      }
+    }
+  });
+}
+
+// ------------------------------------------------------------------------- SpMM, wide N, TMA-staged
+
+// The same row-block x column-slice scheme as k_spmm_wide, with the dense operand's chunks
+// (kWideKC rows x kWideCols columns) brought into shared memory by the tensor-memory
+// accelerator: one thread issues a 2-D bulk tensor copy per chunk into a kTmaStages-deep
+// ring, completion is counted on an mbarrier per stage, and the other threads spend no
+// instructions on staging.  RW (rows per warp) is a template parameter, so no registers or
+// instructions go to unused row slots.  Every wait on an mbarrier is bounded (about a
+// second by the global timer); a wait that gives up sets ERRBIT_TIMEOUT in the status
+// word, the CTA stops computing, lets its issued copies land (again bounded) and returns.
+constexpr int kTmaStages = 3;
+constexpr int kTmaMinN = 256;  // narrower operands take 64-column passes of the small kernel
+
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase with the given parity to complete; false after about `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t a, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+
+// Dense rows per staged chunk: 64, or 56 for fp32 with 8 rows per warp, so that two CTAs
+// (ring + entry buffers) fit in one SM's shared memory.
+template <typename T, int RW>
+constexpr int tma_kc() { return (sizeof(T) == 4 && RW == 8) ? 56 : 64; }
+
+template <typename T, bool TRANS, int RW>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_spmm_tma(const WideArgs<T> A, const __grid_constant__ CUtensorMap tmB) {
+  constexpr int E = (int)sizeof(T);
+  constexpr int KC = tma_kc<T, RW>();
+  constexpr int ROWB = kWideCols * E;  // bytes of one staged dense row
+  constexpr int CHUNK = KC * ROWB;     // bytes of one staged chunk (the TMA box)
+  constexpr int NWARPS = kThreads / 32;
+  extern __shared__ __align__(16) unsigned char s_tx[];  // [kTmaStages][CHUNK] from a 128-byte boundary
+  __shared__ __align__(16) uint2 s_ent[NWARPS][RW][32];
+  __shared__ __align__(8) uint64_t s_full[kTmaStages];
+  __shared__ int s_abort;
+
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  const int64_t r0 = (int64_t)blockIdx.x * (NWARPS * RW);
+  const int n0 = blockIdx.y * kWideCols;
+  const int ncols = min(kWideCols, A.N - n0);
+  const uint32_t full0 = smem_addr(&s_full[0]);
+  const uint32_t xs = (smem_addr(s_tx) + 127u) & ~127u;
+  if (tid == 0) {
+    for (int st = 0; st < kTmaStages; ++st) mbar_init(full0 + 8 * st, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_abort = 0;
+  }
+  __syncthreads();
+  pdl_wait();  // the dense operand may come from the previous grid
+
+  const int64_t nchunks = (A.brows + KC - 1) / KC;
+  auto issue = [&](int64_t ch) {  // thread 0 only
+    const int st = (int)(ch % kTmaStages);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(full0 + 8 * st, (uint32_t)CHUNK);
+    tma_load_2d(xs + st * CHUNK, &tmB, n0, (int)(ch * KC), full0 + 8 * st);
+  };
+  if (tid == 0)
+    for (int64_t ch = 0; ch < kTmaStages - 1 && ch < nchunks; ++ch) issue(ch);
+
+  // entries of the warp's rows, 32 at a time: (col, value bits) in s_ent for broadcast
+  // reads and col in registers for the ballot; (cn, vn) is the prefetched next batch
+  float2 acc[RW][2];
+  int base[RW], end[RW], k[RW], cl[RW], cn[RW];
+  float vn[RW];
+  auto load_batch = [&](int first, int last, int& cc, float& vv) {
+    const int j = first + lane;
+    cc = 0x7fffffff;
+    vv = 0.f;
+    if (j < last) {
+      cc = __ldg(A.idx + j);
+      vv = load1(A.vals + (TRANS ? (int64_t)__ldg(A.perm + j) : (int64_t)j));
+    }
+  };
+  const uint32_t ent0 = smem_addr(&s_ent[wp][0][0]);
+  static_for<0, RW>([&](auto ic) {
+    constexpr int i = decltype(ic)::value;
+    acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+    const int64_t r = r0 + wp * RW + i;
+    const bool valid = r < A.rows;
+    base[i] = valid ? __ldg(A.ptr + r) : 0;
+    end[i] = valid ? __ldg(A.ptr + r + 1) : 0;
+    k[i] = 0;
+    float v0;
+    load_batch(base[i], end[i], cl[i], v0);
+    sts64(ent0 + (i * 32 + lane) * 8, (uint32_t)cl[i], __float_as_uint(v0));
+    load_batch(base[i] + 32, end[i], cn[i], vn[i]);
+  });
+  __syncwarp();
+
+  const uint64_t limit_ns = 1000000000ull;
+  int64_t issued = mn64(kTmaStages - 1, nchunks);  // meaningful in thread 0
+  int64_t ch_stop = nchunks;                        // the chunk whose wait gave up, if any
+  for (int64_t ch = 0; ch < nchunks; ++ch) {
+    if (tid == 0 && issued < nchunks) issue(issued++);  // refills the stage released last round
+    const int st = (int)(ch % kTmaStages);
+    if (!mbar_wait_bounded(full0 + 8 * st, (uint32_t)((ch / kTmaStages) & 1), limit_ns)) s_abort = 1;
+    __syncthreads();
+    if (s_abort) {
+      ch_stop = ch;
+      break;
+    }
+    const int64_t kc = ch * KC;
+    // address of dense row c of this chunk (this lane's 4 columns): xoff + c * ROWB
+    const uint32_t xoff = xs + (uint32_t)(st * CHUNK) + (uint32_t)(lane * 4 * E) - (uint32_t)(kc * ROWB);
+    const int cbound = (int)mn64(kc + KC, A.brows);  // columns below it are staged
+    static_for<0, RW>([&](auto ic) {
+      constexpr int i = decltype(ic)::value;
+      const uint32_t eb = ent0 + i * 32 * 8;
+      while (true) {
+        const int lim = __popc(__ballot_sync(kFull, cl[i] < cbound));  // sorted: a prefix
+        int t = k[i];
+        float2 a01 = acc[i][0], a23 = acc[i][1];
+        auto one = [&](int tt) {
+          const uint2 cv = lds64(eb + tt * 8);
+          const float v = __uint_as_float(cv.y);
+          float4 x;
+          if constexpr (E == 4) {
+            x = lds128(xoff + cv.x * ROWB);
+          } else {
+            const uint2 w = lds64(xoff + cv.x * ROWB);
+            x = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+          }
+          a01 = __ffma2_rn(make_float2(v, v), make_float2(x.x, x.y), a01);
+          a23 = __ffma2_rn(make_float2(v, v), make_float2(x.z, x.w), a23);
+        };
+        for (; t + 4 <= lim; t += 4) {
+          uint2 cv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) cv[u] = lds64(eb + (t + u) * 8);
+          float4 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if constexpr (E == 4) {
+              x[u] = lds128(xoff + cv[u].x * ROWB);
+            } else {
+              const uint2 w = lds64(xoff + cv[u].x * ROWB);
+              x[u] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float v = __uint_as_float(cv[u].y);
+            a01 = __ffma2_rn(make_float2(v, v), make_float2(x[u].x, x[u].y), a01);
+            a23 = __ffma2_rn(make_float2(v, v), make_float2(x[u].z, x[u].w), a23);
+          }
+        }
+        if (t < lim) one(t);
+        if (t + 1 < lim) one(t + 1);
+        if (t + 2 < lim) one(t + 2);
+        acc[i][0] = a01;
+        acc[i][1] = a23;
+        k[i] = lim;
+        if (lim < 32) break;  // the rest of the batch lies beyond this chunk (or the row)
+        base[i] += 32;        // the batch is used up: move to the next one, prefetch the one after
+        cl[i] = cn[i];
+        __syncwarp();
+        sts64(eb + lane * 8, (uint32_t)cn[i], __float_as_uint(vn[i]));
+        __syncwarp();
+        k[i] = 0;
+        load_batch(base[i] + 32, end[i], cn[i], vn[i]);
+      }
+    });
+    __syncthreads();  // every warp is done with this stage before it is refilled
+  }
+  if (ch_stop < nchunks) {  // a wait gave up: report, let the issued copies land (bounded), return
+    if (tid == 0) {
+      if (A.err) atomicOr(A.err, ERRBIT_TIMEOUT);
+      for (int64_t ch = ch_stop; ch < issued; ++ch)
+        mbar_wait_bounded(full0 + 8 * (int)(ch % kTmaStages), (uint32_t)((ch / kTmaStages) & 1), limit_ns);
+    }
+    return;
+  }
+
+  const int c0 = lane * 4;
+  static_for<0, RW>([&](auto ic) {
+    constexpr int i = decltype(ic)::value;
+    const int64_t r = r0 + wp * RW + i;
+    if (r < A.rows && c0 < ncols) {
+      const float a[4] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y};
+      T* dst = A.C + r * A.ldc + n0 + c0;
+      if (c0 + 4 <= ncols && ((uintptr_t)dst % (4 * E)) == 0) {  // one vector store where aligned
+        store_cols<4>(dst, a);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < ncols - c0) store1(dst + j, a[j]);
       }
     }
   });
@@ -917,6 +1148,55 @@ int pick_nc(int ncols, int elem, const void* p0, int64_t ld0, const void* p1, in
   };
   while (nc > 1 && !ok(nc)) nc >>= 1;
   return nc;
+}
+
+// cudaFuncSetAttribute for a kernel's dynamic shared memory above 48 KB, once per device.
+template <auto Kern>
+cudaError_t ensure_dynamic_smem(int bytes) {
+  constexpr int kDev = 64;
+  static std::once_flag once[kDev];
+  static cudaError_t result[kDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kDev) return cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  std::call_once(once[dev], [&] {
+    result[dev] = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  return result[dev];
+}
+
+// The driver's tensor-map encoder, looked up once through the runtime (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map of the dense operand B (brows x N, leading dimension ldb) for boxes of
+// box_rows rows x kWideCols columns; false where TMA's rules (16-byte aligned base and row
+// stride) or the driver rule it out.
+template <typename T>
+bool dense_tensor_map(CUtensorMap* map, const T* B, int64_t brows, int64_t N, int64_t ldb, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr || ((uintptr_t)B % 16) != 0 || ((ldb * (int64_t)sizeof(T)) % 16) != 0) return false;
+  if (brows <= 0 || N <= 0 || brows >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31)) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)brows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ldb * (int64_t)sizeof(T))};
+  const cuuint32_t box[2] = {(cuuint32_t)kWideCols, (cuuint32_t)box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      sizeof(T) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(map, dt, 2, const_cast<T*>(B), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename Args>
@@ -989,18 +1269,16 @@ snk_status spmm_wide(const snk_layout* L, const T* values, const T* B, int64_t N
   A.rows = TRANS ? L->K : L->M;
   A.brows = TRANS ? L->M : L->K;
   A.N = (int)N;
+  A.err = L->err;
   const int64_t slices = (N + kWideCols - 1) / kWideCols;
+  if (slices > 65535) return SNK_ERR_UNSUPPORTED;
   // rows per CTA: 64, halved while the grid would leave SMs idle (at least 8)
   int rb = 8 * kWideRW;
   while (rb > 8 && ((A.rows + rb - 1) / rb) * slices < 3 * (int64_t)L->sm_count) rb /= 2;
   A.rb = rb;
   const dim3 grid((unsigned)((A.rows + rb - 1) / rb), (unsigned)slices);
   const int smem = 2 * kWideKC * kWideCols * (int)sizeof(T);
-  static bool attr_set = false;  // one-time opt-in above 48 KB of dynamic shared memory
-  if (!attr_set) {
-    SNK_CUDA_TRY(cudaFuncSetAttribute(k_spmm_wide<T, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr_set = true;
-  }
+  SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_wide<T, TRANS>>(smem)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
@@ -1015,13 +1293,65 @@ snk_status spmm_wide(const snk_layout* L, const T* values, const T* B, int64_t N
   return SNK_OK;
 }
 
+// The TMA-staged wide kernel; SNK_ERR_UNSUPPORTED (nothing launched) where no tensor map
+// can describe B, so that the caller takes another path.
+template <typename T, bool TRANS>
+snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
+                    cudaStream_t s) {
+  WideArgs<T> A;
+  A.ptr = TRANS ? L->col_ptr : L->row_ptr;
+  A.idx = TRANS ? L->csc_row : L->col;
+  A.perm = TRANS ? L->perm : nullptr;
+  A.vals = values;
+  A.B = B;
+  A.C = C;
+  A.ldb = ldb;
+  A.ldc = ldc;
+  A.rows = TRANS ? L->K : L->M;
+  A.brows = TRANS ? L->M : L->K;
+  A.N = (int)N;
+  A.err = L->err;
+  const int64_t slices = (N + kWideCols - 1) / kWideCols;
+  if (slices > 65535) return SNK_ERR_UNSUPPORTED;
+  // rows per warp: 8, or 4 when 64-row blocks would leave fewer than two CTAs per SM
+  const bool rw8 = ((A.rows + 63) / 64) * slices >= 2 * (int64_t)std::max(L->sm_count, 1);
+  const int rb = rw8 ? 64 : 32;
+  A.rb = rb;
+  const int kc = rw8 ? tma_kc<T, 8>() : tma_kc<T, 4>();
+  CUtensorMap map;
+  if (N >= ((int64_t)1 << 31) || !dense_tensor_map<T>(&map, B, A.brows, N, ldb, kc)) return SNK_ERR_UNSUPPORTED;
+  const int smem = kTmaStages * kc * kWideCols * (int)sizeof(T) + 128;  // + room to align the ring
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((A.rows + rb - 1) / rb), (unsigned)slices);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (rw8) {
+    SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, 8>>(smem)));
+    SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, 8>, A, map)));
+  } else {
+    SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, 4>>(smem)));
+    SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, 4>, A, map)));
+  }
+  return SNK_OK;
+}
+
 template <typename T, bool TRANS>
 snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
                       cudaStream_t s) {
   const int elem = (int)sizeof(T);
   const int64_t rows = TRANS ? L->K : L->M;
-  // very wide operands with 16-byte aligned rows: the row-block x column-slice kernel
-  // (measured faster than 64-column passes of the small kernel from about N = 2048 on)
+  // wide operands: the row-block x column-slice kernels, TMA-staged where a tensor map can
+  // describe B, else staged with cp.async (16-byte aligned rows, from N = kWideMinN)
+  if (N >= kTmaMinN) {
+    const snk_status st = spmm_tma<T, TRANS>(L, values, B, N, ldb, C, ldc, s);
+    if (st != SNK_ERR_UNSUPPORTED) return st;
+  }
   if (N >= kWideMinN && ((uintptr_t)B % 16) == 0 && ((ldb * elem) % 16) == 0 && N < ((int64_t)1 << 31))
     return spmm_wide<T, TRANS>(L, values, B, N, ldb, C, ldc, s);
   for (int64_t col0 = 0; col0 < N; col0 += kCarryCols) {

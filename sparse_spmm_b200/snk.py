@@ -179,6 +179,25 @@ def snk_csr_forward_static(M, K, row_ptr, col, values, X, Y, num_parts=0, stream
               _ld(X), _ptr(Y), _ld(Y), num_parts, _stream(stream)), "snk_csr_forward_static")
 
 
+def snk_sync_status(handle, stream=None):
+    """Synchronise and raise SnkError(SNK_ERR_TIMEOUT) if a product launch gave up a wait."""
+    lib = load_library()
+    lib.snk_sync_status.restype = ctypes.c_int
+    lib.snk_sync_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    _check(lib.snk_sync_status(handle, _stream(stream)), "snk_sync_status")
+
+
+def snk_probe_fp32_fma(blocks, iters, sink, stream=None):
+    """Launch the fp32 FMA-rate probe (a measurement aid); returns its floating-point operations."""
+    lib = load_library()
+    lib.snk_probe_fp32_fma.restype = ctypes.c_int
+    lib.snk_probe_fp32_fma.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    lib.snk_probe_fp32_fma_flops.restype = ctypes.c_int64
+    lib.snk_probe_fp32_fma_flops.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    _check(lib.snk_probe_fp32_fma(blocks, iters, _ptr(sink), _stream(stream)), "snk_probe_fp32_fma")
+    return int(lib.snk_probe_fp32_fma_flops(blocks, iters))
+
+
 # ----------------------------------------------------------------------------- convenience
 
 class Layout:
@@ -253,6 +272,10 @@ class Layout:
         o2n = torch.empty(self.nnz, dtype=torch.int32, device=self.row.device) if want_map else None
         snk_restructure(self.handle, self.values, drop_count, seed, regrow_value, o2n, stream)
         return o2n
+
+    def sync_status(self, stream=None):
+        """Synchronise; raise if a product launch on this layout gave up a bounded wait."""
+        snk_sync_status(self.handle, stream)
 
     # -- inspection
     def arrays(self) -> dict:
