@@ -894,22 +894,37 @@ __global__ void __launch_bounds__(kThreads, 2) k_spmm_wide(const WideArgs<T> A) 
 
 // ------------------------------------------------------------------------- SpMM, wide N, TMA-staged
 
-// The same row-block x column-slice scheme as k_spmm_wide, with the dense operand's chunks
-// (kWideKC rows x kWideCols columns) brought into shared memory by the tensor-memory
-// accelerator: one thread issues a 2-D bulk tensor copy per chunk into a kTmaStages-deep
-// ring, completion is counted on an mbarrier per stage, and the other threads spend no
-// instructions on staging.  RW (rows per warp) is a template parameter, so no registers or
-// instructions go to unused row slots.  Every wait on an mbarrier is bounded (about a
-// second by the global timer); a wait that gives up sets ERRBIT_TIMEOUT in the status
-// word, the CTA stops computing, lets its issued copies land (again bounded) and returns.
+// The row-block x column-slice scheme of k_spmm_wide as a warp-specialised pipeline.  One
+// producer warp brings the dense operand's chunks (KC rows x kWideCols columns) into a
+// kTmaStages-deep shared-memory ring with 2-D bulk tensor copies (TMA); completion is
+// counted on a "full" mbarrier per stage.  Eight consumer warps each own RW rows of the
+// row block and walk every chunk: per row, the entries that fall into the chunk are a
+// prefix of the row's current 32-entry batch (found by a ballot), each broadcast from
+// shared memory as {dense-row byte offset, v, v} so that a lane needs one 16-byte read, one
+// dense-row read and two packed FMAs per entry.  A consumer warp releases a stage by
+// arriving on its "empty" mbarrier; the producer refills a stage once all eight have
+// released it, so no CTA-wide barrier sits in the loop and warps drift up to the ring
+// depth apart.  Every wait is bounded (about a second by the global timer); one that gives
+// up sets ERRBIT_TIMEOUT in the status word, all roles stop, the producer lets its issued
+// copies land (again bounded), and the CTA returns.
 constexpr int kTmaStages = 3;
-constexpr int kTmaMinN = 256;  // narrower operands take 64-column passes of the small kernel
+constexpr int kTmaMinN = 256;     // narrower operands take 64-column passes of the small kernel
+constexpr int kTmaConsumers = 8;  // compute warps; one more warp produces
+constexpr int kTmaThreads = 32 * (kTmaConsumers + 1);
+
+// Dense rows per staged chunk: as many (up to 64) as let two CTAs -- ring plus entry
+// buffers -- share one SM's shared memory.
+template <typename T, int RW>
+constexpr int tma_kc() { return sizeof(T) == 2 ? 64 : (RW >= 8 ? 48 : (RW >= 6 ? 56 : 64)); }
 
 __device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
   uint32_t ok;
@@ -922,7 +937,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
 }
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 // Wait for the phase with the given parity to complete; false after about `limit_ns`.
@@ -941,34 +956,42 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(map), "r"(x), "r"(y), "r"(mbar)
       : "memory");
 }
-
-// Dense rows per staged chunk: 64, or 56 for fp32 with 8 rows per warp, so that two CTAs
-// (ring + entry buffers) fit in one SM's shared memory.
-template <typename T, int RW>
-constexpr int tma_kc() { return (sizeof(T) == 4 && RW == 8) ? 56 : 64; }
+__device__ __forceinline__ uint4 lds128u(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 
 template <typename T, bool TRANS, int RW>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kTmaThreads, 2)
     k_spmm_tma(const WideArgs<T> A, const __grid_constant__ CUtensorMap tmB) {
   constexpr int E = (int)sizeof(T);
   constexpr int KC = tma_kc<T, RW>();
   constexpr int ROWB = kWideCols * E;  // bytes of one staged dense row
   constexpr int CHUNK = KC * ROWB;     // bytes of one staged chunk (the TMA box)
-  constexpr int NWARPS = kThreads / 32;
   extern __shared__ __align__(16) unsigned char s_tx[];  // [kTmaStages][CHUNK] from a 128-byte boundary
-  __shared__ __align__(16) uint2 s_ent[NWARPS][RW][32];
+  __shared__ __align__(16) uint4 s_ent[kTmaConsumers][RW][32];
+  __shared__ int2 s_span[kTmaConsumers][RW];  // per row: {first entry of the current batch, row end}
   __shared__ __align__(8) uint64_t s_full[kTmaStages];
-  __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_empty[kTmaStages];
+  __shared__ volatile int s_abort;
 
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
-  const int64_t r0 = (int64_t)blockIdx.x * (NWARPS * RW);
+  const int64_t r0 = (int64_t)blockIdx.x * (kTmaConsumers * RW);
   const int n0 = blockIdx.y * kWideCols;
   const int ncols = min(kWideCols, A.N - n0);
-  const uint32_t full0 = smem_addr(&s_full[0]);
+  const uint32_t full0 = smem_addr(&s_full[0]), empty0 = smem_addr(&s_empty[0]);
   const uint32_t xs = (smem_addr(s_tx) + 127u) & ~127u;
   if (tid == 0) {
-    for (int st = 0; st < kTmaStages; ++st) mbar_init(full0 + 8 * st, 1);
+    for (int st = 0; st < kTmaStages; ++st) {
+      mbar_init(full0 + 8 * st, 1);
+      mbar_init(empty0 + 8 * st, kTmaConsumers);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_abort = 0;
   }
@@ -976,128 +999,149 @@ __global__ void __launch_bounds__(kThreads, 2)
   pdl_wait();  // the dense operand may come from the previous grid
 
   const int64_t nchunks = (A.brows + KC - 1) / KC;
-  auto issue = [&](int64_t ch) {  // thread 0 only
-    const int st = (int)(ch % kTmaStages);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(full0 + 8 * st, (uint32_t)CHUNK);
-    tma_load_2d(xs + st * CHUNK, &tmB, n0, (int)(ch * KC), full0 + 8 * st);
-  };
-  if (tid == 0)
-    for (int64_t ch = 0; ch < kTmaStages - 1 && ch < nchunks; ++ch) issue(ch);
-
-  // entries of the warp's rows, 32 at a time: (col, value bits) in s_ent for broadcast
-  // reads and col in registers for the ballot; (cn, vn) is the prefetched next batch
-  float2 acc[RW][2];
-  int base[RW], end[RW], k[RW], cl[RW], cn[RW];
-  float vn[RW];
-  auto load_batch = [&](int first, int last, int& cc, float& vv) {
-    const int j = first + lane;
-    cc = 0x7fffffff;
-    vv = 0.f;
-    if (j < last) {
-      cc = __ldg(A.idx + j);
-      vv = load1(A.vals + (TRANS ? (int64_t)__ldg(A.perm + j) : (int64_t)j));
-    }
-  };
-  const uint32_t ent0 = smem_addr(&s_ent[wp][0][0]);
-  static_for<0, RW>([&](auto ic) {
-    constexpr int i = decltype(ic)::value;
-    acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
-    const int64_t r = r0 + wp * RW + i;
-    const bool valid = r < A.rows;
-    base[i] = valid ? __ldg(A.ptr + r) : 0;
-    end[i] = valid ? __ldg(A.ptr + r + 1) : 0;
-    k[i] = 0;
-    float v0;
-    load_batch(base[i], end[i], cl[i], v0);
-    sts64(ent0 + (i * 32 + lane) * 8, (uint32_t)cl[i], __float_as_uint(v0));
-    load_batch(base[i] + 32, end[i], cn[i], vn[i]);
-  });
-  __syncwarp();
-
   const uint64_t limit_ns = 1000000000ull;
-  int64_t issued = mn64(kTmaStages - 1, nchunks);  // meaningful in thread 0
-  int64_t ch_stop = nchunks;                        // the chunk whose wait gave up, if any
-  for (int64_t ch = 0; ch < nchunks; ++ch) {
-    if (tid == 0 && issued < nchunks) issue(issued++);  // refills the stage released last round
-    const int st = (int)(ch % kTmaStages);
-    if (!mbar_wait_bounded(full0 + 8 * st, (uint32_t)((ch / kTmaStages) & 1), limit_ns)) s_abort = 1;
-    __syncthreads();
-    if (s_abort) {
-      ch_stop = ch;
-      break;
+  int64_t issued = 0;  // producer lane: chunks whose copies were issued
+
+  float2 acc[RW][2];
+  if (wp == kTmaConsumers) {
+    // ---- producer
+    if (lane == 0) {
+      for (; issued < nchunks; ++issued) {
+        const int st = (int)(issued % kTmaStages);
+        if (issued >= kTmaStages &&
+            !mbar_wait_bounded(empty0 + 8 * st, (uint32_t)(((issued / kTmaStages) - 1) & 1), limit_ns)) {
+          s_abort = 1;
+          break;
+        }
+        if (s_abort) break;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(full0 + 8 * st, (uint32_t)CHUNK);
+        tma_load_2d(xs + st * CHUNK, &tmB, n0, (int)(issued * KC), full0 + 8 * st);
+      }
     }
-    const int64_t kc = ch * KC;
-    // address of dense row c of this chunk (this lane's 4 columns): xoff + c * ROWB
-    const uint32_t xoff = xs + (uint32_t)(st * CHUNK) + (uint32_t)(lane * 4 * E) - (uint32_t)(kc * ROWB);
-    const int cbound = (int)mn64(kc + KC, A.brows);  // columns below it are staged
+  } else {
+    // ---- consumers: rows r0 + wp*RW + i, i < RW
+    int k[RW], cl[RW];
+    auto load_entry = [&](int first, int last, int& cc, uint4& ent) {
+      const int j = first + lane;
+      cc = 0x7fffffff;
+      ent = make_uint4(0u, 0u, 0u, 0u);
+      if (j < last) {
+        cc = __ldg(A.idx + j);
+        const float v = load1(A.vals + (TRANS ? (int64_t)__ldg(A.perm + j) : (int64_t)j));
+        ent = make_uint4((uint32_t)cc * (uint32_t)ROWB, __float_as_uint(v), __float_as_uint(v), 0u);
+      }
+    };
+    auto prefetch_next = [&](int first, int last) {  // the batch after this one, into L1
+      const int j = first + 32 + lane;
+      if (j < last) {
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(A.idx + j));
+        if (TRANS) asm volatile("prefetch.global.L1 [%0];" ::"l"(A.perm + j));
+      }
+    };
+    const uint32_t ent0 = smem_addr(&s_ent[wp][0][0]);
     static_for<0, RW>([&](auto ic) {
       constexpr int i = decltype(ic)::value;
-      const uint32_t eb = ent0 + i * 32 * 8;
-      while (true) {
-        const int lim = __popc(__ballot_sync(kFull, cl[i] < cbound));  // sorted: a prefix
-        int t = k[i];
+      acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+      const int64_t r = r0 + wp * RW + i;
+      const bool valid = r < A.rows;
+      const int rbeg = valid ? __ldg(A.ptr + r) : 0;
+      const int rend = valid ? __ldg(A.ptr + r + 1) : 0;
+      if (lane == 0) s_span[wp][i] = make_int2(rbeg, rend);
+      k[i] = 0;
+      uint4 ent;
+      load_entry(rbeg, rend, cl[i], ent);
+      sts128u(ent0 + (i * 32 + lane) * 16, ent);
+      prefetch_next(rbeg, rend);
+    });
+    __syncwarp();
+
+    const uint32_t lane_off = (uint32_t)(lane * 4 * E);
+    for (int64_t ch = 0; ch < nchunks; ++ch) {
+      const int st = (int)(ch % kTmaStages);
+      bool ok = s_abort == 0 && mbar_wait_bounded(full0 + 8 * st, (uint32_t)((ch / kTmaStages) & 1), limit_ns);
+      ok = __all_sync(kFull, ok);
+      if (!ok) {
+        if (lane == 0) s_abort = 1;
+        break;
+      }
+      const int64_t kc = ch * KC;
+      // dense row c of this chunk (this lane's 4 columns) sits at xoff + c * ROWB
+      const uint32_t xoff = xs + (uint32_t)(st * CHUNK) + lane_off - (uint32_t)(kc * ROWB);
+      const int cbound = (int)mn64(kc + KC, A.brows);  // columns below it are staged
+      static_for<0, RW>([&](auto ic) {
+        constexpr int i = decltype(ic)::value;
+        const uint32_t eb = ent0 + i * 32 * 16;
         float2 a01 = acc[i][0], a23 = acc[i][1];
-        auto one = [&](int tt) {
-          const uint2 cv = lds64(eb + tt * 8);
-          const float v = __uint_as_float(cv.y);
-          float4 x;
-          if constexpr (E == 4) {
-            x = lds128(xoff + cv.x * ROWB);
-          } else {
-            const uint2 w = lds64(xoff + cv.x * ROWB);
-            x = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-          }
-          a01 = __ffma2_rn(make_float2(v, v), make_float2(x.x, x.y), a01);
-          a23 = __ffma2_rn(make_float2(v, v), make_float2(x.z, x.w), a23);
+        auto fma_x = [&](const uint4& e, const float4& x) {
+          const float2 vv = make_float2(__uint_as_float(e.y), __uint_as_float(e.z));
+          a01 = __ffma2_rn(vv, make_float2(x.x, x.y), a01);
+          a23 = __ffma2_rn(vv, make_float2(x.z, x.w), a23);
         };
-        for (; t + 4 <= lim; t += 4) {
-          uint2 cv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) cv[u] = lds64(eb + (t + u) * 8);
-          float4 x[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if constexpr (E == 4) {
-              x[u] = lds128(xoff + cv[u].x * ROWB);
-            } else {
-              const uint2 w = lds64(xoff + cv[u].x * ROWB);
-              x[u] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-            }
+        auto load_x = [&](const uint4& e) -> float4 {
+          if constexpr (E == 4) {
+            return lds128(xoff + e.x);
+          } else {
+            const uint2 w = lds64(xoff + e.x);
+            return make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
           }
+        };
+        while (true) {
+          const int lim = __popc(__ballot_sync(kFull, cl[i] < cbound));  // sorted: a prefix
+          int t = k[i];
+          for (; t + 4 <= lim; t += 4) {
+            uint4 e[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float v = __uint_as_float(cv[u].y);
-            a01 = __ffma2_rn(make_float2(v, v), make_float2(x[u].x, x[u].y), a01);
-            a23 = __ffma2_rn(make_float2(v, v), make_float2(x[u].z, x[u].w), a23);
+            for (int u = 0; u < 4; ++u) e[u] = lds128u(eb + (t + u) * 16);
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = load_x(e[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) fma_x(e[u], x[u]);
           }
+          if (t < lim) {  // up to three more: loads first (a spent slot re-reads entry t), FMAs predicated
+            uint4 e[3];
+            float4 x[3];
+#pragma unroll
+            for (int u = 0; u < 3; ++u) e[u] = lds128u(eb + (t + u < lim ? t + u : t) * 16);
+#pragma unroll
+            for (int u = 0; u < 3; ++u) x[u] = load_x(e[u]);
+            fma_x(e[0], x[0]);
+            if (t + 1 < lim) fma_x(e[1], x[1]);
+            if (t + 2 < lim) fma_x(e[2], x[2]);
+          }
+          k[i] = lim;
+          if (lim < 32) break;  // the rest of the batch lies beyond this chunk (or the row)
+          // the batch is used up: load the next one (prefetched into L1) and the one after
+          const int2 sp = s_span[wp][i];
+          const int nb = sp.x + 32;
+          uint4 ent;
+          load_entry(nb, sp.y, cl[i], ent);
+          __syncwarp();
+          sts128u(eb + lane * 16, ent);
+          if (lane == 0) s_span[wp][i].x = nb;
+          __syncwarp();
+          k[i] = 0;
+          prefetch_next(nb, sp.y);
         }
-        if (t < lim) one(t);
-        if (t + 1 < lim) one(t + 1);
-        if (t + 2 < lim) one(t + 2);
         acc[i][0] = a01;
         acc[i][1] = a23;
-        k[i] = lim;
-        if (lim < 32) break;  // the rest of the batch lies beyond this chunk (or the row)
-        base[i] += 32;        // the batch is used up: move to the next one, prefetch the one after
-        cl[i] = cn[i];
-        __syncwarp();
-        sts64(eb + lane * 8, (uint32_t)cn[i], __float_as_uint(vn[i]));
-        __syncwarp();
-        k[i] = 0;
-        load_batch(base[i] + 32, end[i], cn[i], vn[i]);
-      }
-    });
-    __syncthreads();  // every warp is done with this stage before it is refilled
+      });
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * st);  // this warp is done with the stage
+    }
   }
-  if (ch_stop < nchunks) {  // a wait gave up: report, let the issued copies land (bounded), return
-    if (tid == 0) {
+  __syncthreads();  // every role has finished (all waits above are bounded)
+  if (s_abort) {    // a wait gave up: report, let the issued copies land (bounded), return
+    if (wp == kTmaConsumers && lane == 0) {
       if (A.err) atomicOr(A.err, ERRBIT_TIMEOUT);
-      for (int64_t ch = ch_stop; ch < issued; ++ch)
+      // the last phase issued into each stage (earlier ones completed before it was reissued)
+      for (int64_t ch = mn64(issued, nchunks) - 1; ch >= 0 && ch >= issued - kTmaStages; --ch)
         mbar_wait_bounded(full0 + 8 * (int)(ch % kTmaStages), (uint32_t)((ch / kTmaStages) & 1), limit_ns);
     }
     return;
   }
+  if (wp == kTmaConsumers) return;
 
   const int c0 = lane * 4;
   static_for<0, RW>([&](auto ic) {
@@ -1295,6 +1339,28 @@ snk_status spmm_wide(const snk_layout* L, const T* values, const T* B, int64_t N
 
 // The TMA-staged wide kernel; SNK_ERR_UNSUPPORTED (nothing launched) where no tensor map
 // can describe B, so that the caller takes another path.
+template <typename T, bool TRANS, int RW>
+snk_status launch_tma(const WideArgs<T>& A, const T* B, int64_t N, int64_t ldb, int64_t slices, cudaStream_t s) {
+  constexpr int kc = tma_kc<T, RW>();
+  CUtensorMap map;
+  if (!dense_tensor_map<T>(&map, B, A.brows, N, ldb, kc)) return SNK_ERR_UNSUPPORTED;
+  const int smem = kTmaStages * kc * kWideCols * (int)sizeof(T) + 128;  // + room to align the ring
+  const int rb = kTmaConsumers * RW;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((A.rows + rb - 1) / rb), (unsigned)slices);
+  cfg.blockDim = dim3(kTmaThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, RW>>(smem)));
+  SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, RW>, A, map)));
+  return SNK_OK;
+}
+
 template <typename T, bool TRANS>
 snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
                     cudaStream_t s) {
@@ -1311,34 +1377,25 @@ snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N,
   A.brows = TRANS ? L->M : L->K;
   A.N = (int)N;
   A.err = L->err;
+  A.rb = 0;
   const int64_t slices = (N + kWideCols - 1) / kWideCols;
-  if (slices > 65535) return SNK_ERR_UNSUPPORTED;
-  // rows per warp: 8, or 4 when 64-row blocks would leave fewer than two CTAs per SM
-  const bool rw8 = ((A.rows + 63) / 64) * slices >= 2 * (int64_t)std::max(L->sm_count, 1);
-  const int rb = rw8 ? 64 : 32;
-  A.rb = rb;
-  const int kc = rw8 ? tma_kc<T, 8>() : tma_kc<T, 4>();
-  CUtensorMap map;
-  if (N >= ((int64_t)1 << 31) || !dense_tensor_map<T>(&map, B, A.brows, N, ldb, kc)) return SNK_ERR_UNSUPPORTED;
-  const int smem = kTmaStages * kc * kWideCols * (int)sizeof(T) + 128;  // + room to align the ring
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((A.rows + rb - 1) / rb), (unsigned)slices);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (rw8) {
-    SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, 8>>(smem)));
-    SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, 8>, A, map)));
-  } else {
-    SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, 4>>(smem)));
-    SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, 4>, A, map)));
+  if (N >= ((int64_t)1 << 31) || slices > 65535) return SNK_ERR_UNSUPPORTED;
+  // rows per consumer warp: the choice among 8, 6 and 4 with the shortest estimated
+  // makespan, rounds of two CTAs per SM x (rows per warp + a staging term)
+  const int64_t slots = 2 * (int64_t)std::max(L->sm_count, 1);
+  int best = 8;
+  int64_t best_cost = -1;
+  for (int rw : {8, 6, 4}) {
+    const int64_t tiles = ((A.rows + 8 * rw - 1) / (8 * rw)) * slices;
+    const int64_t cost = ((tiles + slots - 1) / slots) * (rw + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = rw;
+    }
   }
-  return SNK_OK;
+  if (best == 8) return launch_tma<T, TRANS, 8>(A, B, N, ldb, slices, s);
+  if (best == 6) return launch_tma<T, TRANS, 6>(A, B, N, ldb, slices, s);
+  return launch_tma<T, TRANS, 4>(A, B, N, ldb, slices, s);
 }
 
 template <typename T, bool TRANS>

@@ -48,12 +48,14 @@ def test_wide_operands(dtype, N, pad):
     L.sync_status()
 
 
+# shapes whose grids make the launcher pick 8 (4096 x 3000, N = 512: one round of 64-row
+# blocks) and 6 (2500 x 600, N = 2048) rows per consumer warp on a 148-SM GPU
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_wide_eight_rows_per_warp(dtype):
-    # enough 64-row blocks x slices for two CTAs per SM: the 8-rows-per-warp variant
-    layer = wl.uniform_layer(2500, 600, 0.9, dtype, 5, "W")
+@pytest.mark.parametrize("M,K,N", [(4096, 3000, 512), (2500, 600, 2048)])
+def test_wide_rows_per_warp_variants(dtype, M, K, N):
+    layer = wl.uniform_layer(M, K, 0.95, dtype, 5, "W")
     L = gpu_layout(layer)
     ref = check_build(L, layer)
-    rows = np.unique(np.concatenate([np.arange(0, 2500, 37), [2499]]))
-    check_products(layer, ref, L, 2048, seed=4, ops=("forward", "backward_input"), sample_rows=rows)
+    rows = np.unique(np.concatenate([np.arange(0, M, 37), [M - 1, K - 1]]))
+    check_products(layer, ref, L, N, seed=4, ops=("forward", "backward_input"), sample_rows=rows)
     L.sync_status()
