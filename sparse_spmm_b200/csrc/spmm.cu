@@ -681,21 +681,13 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
 
 // ------------------------------------------------------------------------- SpMM, wide N
 
-// For wide dense operands (N > kCarryCols) the work splits over (row block, column slice)
-// pairs instead of nnz parts: each CTA owns whole output rows, so no row is ever split,
-// and row skew is amortised by the many column slices.  The dense operand's slice is
-// staged through shared memory in chunks of kWideKC rows with double-buffered cp.async,
-// so every staged element serves all rows of the block that hold its column.  Each warp
-// keeps kWideRW rows' accumulators in registers and walks each row's column-sorted
-// entries chunk by chunk: entries arrive in coalesced batches of 32 (the next batch is
-// prefetched), one warp ballot counts how many of them fall inside the current chunk,
-// and those are consumed four at a time (independent shared-memory reads, then packed
-// FMAs).  Every lane owns four columns (kWideCols = 128 per slice).  The bound is the
-// shared-memory read of one operand element per FMA.
-constexpr int kWideCols = 128;   // columns per slice (4 per lane)
-constexpr int kWideKC = 64;      // dense rows per staged chunk
-constexpr int kWideRW = 8;       // rows per warp (row block <= 64 rows)
-constexpr int kWideMinN = 2048;  // narrower operands take 64-column passes of the small kernel
+// For wide dense operands the work splits over (row block, column slice) pairs instead of
+// nnz parts: each CTA owns whole output rows, so no row is ever split, and row skew is
+// amortised by the many column slices.  The dense operand's slice is staged through shared
+// memory in chunks of dense rows, so every staged element serves all rows of the block that
+// hold its column.  Every lane owns four columns (kWideCols = 128 per slice).  The bound is
+// the shared-memory read of one operand element per FMA.
+constexpr int kWideCols = 128;  // columns per slice (4 per lane)
 
 template <typename T>
 struct WideArgs {
@@ -708,17 +700,8 @@ struct WideArgs {
   int64_t ldb, ldc;
   int64_t rows, brows;
   int N;
-  int rb;               // rows per CTA (8 * rows per warp, <= 8 * kWideRW)
   uint32_t* err;        // status word (may be null): ERRBIT_TIMEOUT if a pipeline wait gave up
 };
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ float4 lds128(uint32_t a) {
@@ -731,170 +714,10 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
   return v;
 }
-__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
-}
-
-template <typename T, bool TRANS>
-__global__ void __launch_bounds__(kThreads, 2) k_spmm_wide(const WideArgs<T> A) {
-  constexpr int E = (int)sizeof(T);
-  constexpr int RB_BYTES = kWideCols * E;          // bytes of one staged dense row
-  constexpr int CHUNK = kWideKC * RB_BYTES;        // bytes of one staged chunk
-  extern __shared__ __align__(16) unsigned char s_x[];  // [2][CHUNK]
-  // per warp and row: the current batch of 32 (col, value bits) pairs, read by broadcast
-  __shared__ __align__(16) uint2 s_ent[kThreads / 32][kWideRW][32];
-
-  pdl_launch_dependents();
-  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
-  const int64_t r0 = (int64_t)blockIdx.x * A.rb;
-  const int n0 = blockIdx.y * kWideCols;
-  const int ncols = min(kWideCols, A.N - n0);
-  const int rw = A.rb / 8;  // rows of this warp: r0 + wp*rw + i, i < rw
-  pdl_wait();
-
-  // chunk staging: CHUNK / 16 pieces of 16 bytes, spread over the CTA
-  auto stage = [&](int buf, int64_t kc) {
-    constexpr int PIECES = CHUNK / 16;
-    constexpr int PER_ROW = RB_BYTES / 16;
-    unsigned char* dst = s_x + buf * CHUNK;
-    for (int q = tid; q < PIECES; q += kThreads) {
-      const int rr = q / PER_ROW, cb = (q % PER_ROW) * 16;  // row in chunk, byte in row
-      const int64_t brow = kc + rr;
-      const int col_e = cb / E;  // first element of the piece within the slice
-      int bytes = 0;
-      const T* src = A.B;
-      if (brow < A.brows && col_e < ncols) {
-        bytes = min(16, (ncols - col_e) * E);
-        src = A.B + brow * A.ldb + n0 + col_e;
-      }
-      cp_async16(dst + rr * RB_BYTES + cb, src, bytes);
-    }
-  };
-
-  // per row i: entries [base, end); the current batch holds entries base .. base+31
-  // (col = INT_MAX past the end) in registers (cl, for the ballot) and in s_ent (for the
-  // broadcast reads); slots < k are consumed; (cn, vn) is the prefetched next batch.
-  float acc[kWideRW][4];
-  int base[kWideRW], end[kWideRW], k[kWideRW];
-  int cl[kWideRW], cn[kWideRW];
-  float vn[kWideRW];
-  auto load_batch = [&](int first, int last, int& cc, float& vv) {
-    const int j = first + lane;
-    cc = 0x7fffffff;
-    vv = 0.f;
-    if (j < last) {
-      cc = __ldg(A.idx + j);
-      vv = load1(A.vals + (TRANS ? (int64_t)__ldg(A.perm + j) : (int64_t)j));
-    }
-  };
-  const uint32_t ent0 = smem_addr(&s_ent[wp][0][0]);
-  static_for<0, kWideRW>([&](auto ic) {
-    constexpr int i = decltype(ic)::value;
-    acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    const int64_t r = r0 + wp * rw + i;
-    const bool valid = i < rw && r < A.rows;
-    base[i] = valid ? __ldg(A.ptr + r) : 0;
-    end[i] = valid ? __ldg(A.ptr + r + 1) : 0;
-    k[i] = 0;
-    float v0;
-    load_batch(base[i], end[i], cl[i], v0);
-    sts64(ent0 + (i * 32 + lane) * 8, (uint32_t)cl[i], __float_as_uint(v0));
-    load_batch(base[i] + 32, end[i], cn[i], vn[i]);
-  });
-  __syncwarp();
-
-  const int64_t nchunks = (A.brows + kWideKC - 1) / kWideKC;
-  const uint32_t xs0 = smem_addr(s_x) + lane * 4 * E;
-  stage(0, 0);
-  cp_async_commit();
-  for (int64_t ch = 0; ch < nchunks; ++ch) {
-    const int64_t kc = ch * kWideKC;
-    if (ch + 1 < nchunks) stage((int)((ch + 1) & 1), kc + kWideKC);
-    cp_async_commit();
-    cp_async_wait_1();
-    __syncthreads();
-    // address of dense row c of this chunk (this lane's 4 columns): xoff + c * RB_BYTES
-    const uint32_t xoff = xs0 + (uint32_t)((ch & 1) * CHUNK) - (uint32_t)(kc * RB_BYTES);
-    const int kend = (int)min((int64_t)kWideKC, A.brows - kc);
-    const int cbound = (int)kc + kend;  // columns below this are in the staged chunk
-    static_for<0, kWideRW>([&](auto ic) {
-      constexpr int i = decltype(ic)::value;
-      const uint32_t eb = ent0 + i * 32 * 8;
-      while (true) {
-        const int lim = __popc(__ballot_sync(kFull, cl[i] < cbound));  // sorted: a prefix
-        int t = k[i];
-        float2 a01 = make_float2(acc[i][0], acc[i][1]), a23 = make_float2(acc[i][2], acc[i][3]);
-        for (; t + 4 <= lim; t += 4) {  // full groups of four entries
-          float4 x[4];
-          float v[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint2 cv = lds64(eb + (t + u) * 8);
-            v[u] = __uint_as_float(cv.y);
-            if constexpr (E == 4) {
-              x[u] = lds128(xoff + cv.x * RB_BYTES);
-            } else {
-              const uint2 w = lds64(xoff + cv.x * RB_BYTES);
-              x[u] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            a01 = __ffma2_rn(make_float2(v[u], v[u]), make_float2(x[u].x, x[u].y), a01);
-            a23 = __ffma2_rn(make_float2(v[u], v[u]), make_float2(x[u].z, x[u].w), a23);
-          }
-        }
-        for (; t < lim; ++t) {  // the rest, one at a time
-          const uint2 cv = lds64(eb + t * 8);
-          const float v = __uint_as_float(cv.y);
-          float4 x;
-          if constexpr (E == 4) {
-            x = lds128(xoff + cv.x * RB_BYTES);
-          } else {
-            const uint2 w = lds64(xoff + cv.x * RB_BYTES);
-            x = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-          }
-          a01 = __ffma2_rn(make_float2(v, v), make_float2(x.x, x.y), a01);
-          a23 = __ffma2_rn(make_float2(v, v), make_float2(x.z, x.w), a23);
-        }
-        acc[i][0] = a01.x; acc[i][1] = a01.y; acc[i][2] = a23.x; acc[i][3] = a23.y;
-        k[i] = max(k[i], lim);
-        if (lim < 32) break;  // the rest of the batch lies beyond this chunk (or the row)
-        // the batch is used up: move to the next one and prefetch the one after
-        base[i] += 32;
-        cl[i] = cn[i];
-        __syncwarp();
-        sts64(eb + lane * 8, (uint32_t)cn[i], __float_as_uint(vn[i]));
-        __syncwarp();
-        k[i] = 0;
-        load_batch(base[i] + 32, end[i], cn[i], vn[i]);
-      }
-    });
-    __syncthreads();
-  }
-  cp_async_wait_0();
-
-  // write the rows: lane owns columns n0 + 4 lane .. + 3
-  const int c0 = lane * 4;
-  static_for<0, kWideRW>([&](auto ic) {
-    constexpr int i = decltype(ic)::value;
-    const int64_t r = r0 + wp * rw + i;
-    if (i < rw && r < A.rows && c0 < ncols) {
-      T* dst = A.C + r * A.ldc + n0 + c0;
-      if (c0 + 4 <= ncols && ((uintptr_t)dst % (4 * E)) == 0) {  // one vector store where aligned
-        store_cols<4>(dst, acc[i]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (j < ncols - c0) store1(dst + j, acc[i][j]);
-      }
-    }
-  });
-}
 
 // ------------------------------------------------------------------------- SpMM, wide N, TMA-staged
 
-// The row-block x column-slice scheme of k_spmm_wide as a warp-specialised pipeline.  One
+// The row-block x column-slice kernel, as a warp-specialised pipeline.  One
 // producer warp brings the dense operand's chunks (KC rows x kWideCols columns) into a
 // kTmaStages-deep shared-memory ring with 2-D bulk tensor copies (TMA); completion is
 // counted on a "full" mbarrier per stage.  Eight consumer warps each own RW rows of the
@@ -1298,45 +1121,6 @@ SddmmKernel<T> pick_sddmm(int nc, int g) {
   return nullptr;
 }
 
-template <typename T, bool TRANS>
-snk_status spmm_wide(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
-                     cudaStream_t s) {
-  WideArgs<T> A;
-  A.ptr = TRANS ? L->col_ptr : L->row_ptr;
-  A.idx = TRANS ? L->csc_row : L->col;
-  A.perm = TRANS ? L->perm : nullptr;
-  A.vals = values;
-  A.B = B;
-  A.C = C;
-  A.ldb = ldb;
-  A.ldc = ldc;
-  A.rows = TRANS ? L->K : L->M;
-  A.brows = TRANS ? L->M : L->K;
-  A.N = (int)N;
-  A.err = L->err;
-  const int64_t slices = (N + kWideCols - 1) / kWideCols;
-  if (slices > 65535) return SNK_ERR_UNSUPPORTED;
-  // rows per CTA: 64, halved while the grid would leave SMs idle (at least 8)
-  int rb = 8 * kWideRW;
-  while (rb > 8 && ((A.rows + rb - 1) / rb) * slices < 3 * (int64_t)L->sm_count) rb /= 2;
-  A.rb = rb;
-  const dim3 grid((unsigned)((A.rows + rb - 1) / rb), (unsigned)slices);
-  const int smem = 2 * kWideKC * kWideCols * (int)sizeof(T);
-  SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_wide<T, TRANS>>(smem)));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  SNK_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_spmm_wide<T, TRANS>, A));
-  return SNK_OK;
-}
-
 // The TMA-staged wide kernel; SNK_ERR_UNSUPPORTED (nothing launched) where no tensor map
 // can describe B, so that the caller takes another path.
 template <typename T, bool TRANS, int RW>
@@ -1377,7 +1161,6 @@ snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N,
   A.brows = TRANS ? L->M : L->K;
   A.N = (int)N;
   A.err = L->err;
-  A.rb = 0;
   const int64_t slices = (N + kWideCols - 1) / kWideCols;
   if (N >= ((int64_t)1 << 31) || slices > 65535) return SNK_ERR_UNSUPPORTED;
   // rows per consumer warp: the choice among 8, 6 and 4 with the shortest estimated
@@ -1403,14 +1186,12 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
                       cudaStream_t s) {
   const int elem = (int)sizeof(T);
   const int64_t rows = TRANS ? L->K : L->M;
-  // wide operands: the row-block x column-slice kernels, TMA-staged where a tensor map can
-  // describe B, else staged with cp.async (16-byte aligned rows, from N = kWideMinN)
+  // wide operands: the TMA-staged row-block x column-slice kernel where a tensor map can
+  // describe B (16-byte aligned base and row stride)
   if (N >= kTmaMinN) {
     const snk_status st = spmm_tma<T, TRANS>(L, values, B, N, ldb, C, ldc, s);
     if (st != SNK_ERR_UNSUPPORTED) return st;
   }
-  if (N >= kWideMinN && ((uintptr_t)B % 16) == 0 && ((ldb * elem) % 16) == 0 && N < ((int64_t)1 << 31))
-    return spmm_wide<T, TRANS>(L, values, B, N, ldb, C, ldc, s);
   for (int64_t col0 = 0; col0 < N; col0 += kCarryCols) {
     const int ncols = (int)std::min<int64_t>(kCarryCols, N - col0);
     const T* Bc = B + col0;
