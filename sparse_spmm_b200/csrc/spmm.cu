@@ -723,7 +723,7 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
 // counted on a "full" mbarrier per stage.  Eight consumer warps each own RW rows of the
 // row block and walk every chunk: per row, the entries that fall into the chunk are a
 // prefix of the row's current 32-entry batch (found by a ballot), each broadcast from
-// shared memory as {dense-row byte offset, v, v} so that a lane needs one 16-byte read, one
+// shared memory as {v, v, dense-row byte offset} so that a lane needs one 16-byte read, one
 // dense-row read and two packed FMAs per entry.  A consumer warp releases a stage by
 // arriving on its "empty" mbarrier; the producer refills a stage once all eight have
 // released it, so no CTA-wide barrier sits in the loop and warps drift up to the ring
@@ -797,7 +797,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
   constexpr int ROWB = kWideCols * E;  // bytes of one staged dense row
   constexpr int CHUNK = KC * ROWB;     // bytes of one staged chunk (the TMA box)
   extern __shared__ __align__(16) unsigned char s_tx[];  // [kTmaStages][CHUNK] from a 128-byte boundary
-  __shared__ __align__(16) uint4 s_ent[kTmaConsumers][RW][32];
+  __shared__ __align__(16) uint4 s_ent[kTmaConsumers][RW][32];  // {v, v, dense-row byte offset, 0}
   __shared__ int2 s_span[kTmaConsumers][RW];  // per row: {first entry of the current batch, row end}
   __shared__ __align__(8) uint64_t s_full[kTmaStages];
   __shared__ __align__(8) uint64_t s_empty[kTmaStages];
@@ -852,7 +852,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
       if (j < last) {
         cc = __ldg(A.idx + j);
         const float v = load1(A.vals + (TRANS ? (int64_t)__ldg(A.perm + j) : (int64_t)j));
-        ent = make_uint4((uint32_t)cc * (uint32_t)ROWB, __float_as_uint(v), __float_as_uint(v), 0u);
+        ent = make_uint4(__float_as_uint(v), __float_as_uint(v), (uint32_t)cc * (uint32_t)ROWB, 0u);
       }
     };
     auto prefetch_next = [&](int first, int last) {  // the batch after this one, into L1
@@ -897,15 +897,15 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
         const uint32_t eb = ent0 + i * 32 * 16;
         float2 a01 = acc[i][0], a23 = acc[i][1];
         auto fma_x = [&](const uint4& e, const float4& x) {
-          const float2 vv = make_float2(__uint_as_float(e.y), __uint_as_float(e.z));
+          const float2 vv = make_float2(__uint_as_float(e.x), __uint_as_float(e.y));
           a01 = __ffma2_rn(vv, make_float2(x.x, x.y), a01);
           a23 = __ffma2_rn(vv, make_float2(x.z, x.w), a23);
         };
         auto load_x = [&](const uint4& e) -> float4 {
           if constexpr (E == 4) {
-            return lds128(xoff + e.x);
+            return lds128(xoff + e.z);
           } else {
-            const uint2 w = lds64(xoff + e.x);
+            const uint2 w = lds64(xoff + e.z);
             return make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
           }
         };
@@ -922,16 +922,23 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
 #pragma unroll
             for (int u = 0; u < 4; ++u) fma_x(e[u], x[u]);
           }
-          if (t < lim) {  // up to three more: loads first (a spent slot re-reads entry t), FMAs predicated
+          if (t < lim) {  // up to three more: predicated loads first, then the FMAs
             uint4 e[3];
             float4 x[3];
 #pragma unroll
-            for (int u = 0; u < 3; ++u) e[u] = lds128u(eb + (t + u < lim ? t + u : t) * 16);
+            for (int u = 0; u < 3; ++u) {
+              e[u] = make_uint4(0u, 0u, 0u, 0u);
+              x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-            for (int u = 0; u < 3; ++u) x[u] = load_x(e[u]);
-            fma_x(e[0], x[0]);
-            if (t + 1 < lim) fma_x(e[1], x[1]);
-            if (t + 2 < lim) fma_x(e[2], x[2]);
+            for (int u = 0; u < 3; ++u)
+              if (t + u < lim) e[u] = lds128u(eb + (t + u) * 16);
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+              if (t + u < lim) x[u] = load_x(e[u]);
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+              if (t + u < lim) fma_x(e[u], x[u]);
           }
           k[i] = lim;
           if (lim < 32) break;  // the rest of the batch lies beyond this chunk (or the row)
