@@ -44,14 +44,15 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 # ----------------------------------------------------------------------------- byte / flop model
 
-def op_bytes(op: str, M: int, K: int, nnz: int, N: int, s: int) -> int:
-    """Algorithmic bytes of one op: compulsory traffic, int32 indices, dense operands once."""
+def op_bytes(op: str, M: int, K: int, nnz: int, N: int, s: int, ib: int = 4) -> int:
+    """Algorithmic bytes of one op: compulsory traffic, dense operands once; ib = bytes of a
+    column / row index (4 as the format specifies, 2 with 16-bit indices; perm stays 4)."""
     if op == "forward":
-        return nnz * (s + 4) + 4 * (M + 1) + K * N * s + M * N * s
+        return nnz * (s + ib) + 4 * (M + 1) + K * N * s + M * N * s
     if op == "backward_input":
-        return nnz * (s + 4 + 4) + 4 * (K + 1) + M * N * s + K * N * s
+        return nnz * (s + ib + 4) + 4 * (K + 1) + M * N * s + K * N * s
     if op == "backward_weight":
-        return nnz * (4 + s) + 4 * (M + 1) + K * N * s + M * N * s
+        return nnz * (ib + s) + 4 * (M + 1) + K * N * s + M * N * s
     raise ValueError(op)
 
 
@@ -252,30 +253,48 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
     torch.cuda.synchronize()
 
     # per-op graphs: R launches of one (op, N), to time each kernel alone (L2-cold)
-    per_op = {}
     reps = 20
-    for N in batches:
-        for op in OPS:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for c in copies:
-                    launch(c, op, N, stream)
-            with torch.cuda.stream(stream):
-                g.replay()
-            stream.synchronize()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                e0.record(stream)
-                for _ in range(reps):
+
+    def time_ops(ib: int) -> dict:
+        res = {}
+        for N in batches:
+            for op in OPS:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for c in copies:
+                        launch(c, op, N, stream)
+                with torch.cuda.stream(stream):
                     g.replay()
-                e1.record(stream)
-            e1.synchronize()
-            us = e0.elapsed_time(e1) * 1e3 / (reps * R)
-            b = op_bytes(op, M, K, nnz, N, s)
-            per_op[f"{op}@N={N}"] = {"us": round(us, 3), "bytes": b, "gbs": round(b / us / 1e3, 1),
-                                     "gflops": round(op_flops(nnz, N) / us / 1e3, 1)}
-            del g
+                stream.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                e1.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / (reps * R)
+                b = op_bytes(op, M, K, nnz, N, s, ib)
+                res[f"{op}@N={N}"] = {"us": round(us, 3), "bytes": b, "gbs": round(b / us / 1e3, 1),
+                                      "gflops": round(op_flops(nnz, N) / us / 1e3, 1)}
+                del g
+        return res
+
+    per_op = time_ops(4)
+    # the same ops reading 16-bit column / row indices (bit-identical results), with their
+    # own byte model; the step above and the headline use the int32 format
+    for c in copies:
+        c["L"].set_index_bits(16)
+    per_op16 = time_ops(2)
+    for c in copies:
+        c["L"].set_index_bits(32)
+    us32 = sum(v["us"] for v in per_op.values())
+    us16 = sum(v["us"] for v in per_op16.values())
+    index16 = {"ops_us_sum": round(us16, 3), "int32_ops_us_sum": round(us32, 3),
+               "time_ratio_vs_int32": round(us16 / us32, 4),
+               "gbs_own_model": round(sum(v["bytes"] for v in per_op16.values()) / us16 / 1e3, 1),
+               "byte_model": "col / csc_row 2 B per nonzero, perm 4 B", "per_op_us": {k: v["us"] for k, v in per_op16.items()}}
 
     # warm-up of the step graphs, then the timed region
     with torch.cuda.stream(stream):
@@ -378,6 +397,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
         "clocks": clk.summary(),
         "gpu_launches": launches_per_step * args.steps,
         "per_op": per_op,
+        "index16": index16,
         "preprocess": {"build_ms": round(t_build * 1e3, 3), "restructure_ms": round(t_rs * 1e3, 3),
                        "restructure_drop": nnz // 10, "note": "host wall clock incl. the one status sync"},
     }
@@ -492,8 +512,8 @@ def run_reference(args, rank: int, world: int) -> dict:
 
 
 def run_profile(args) -> None:
-    """Two passes of the step's launches on one layout, no timing: pass 0 warms up, pass 1 is
-    what an ncu capture selects (-s 3*len(batches) -c 3*len(batches)).  For profiling only."""
+    """Two passes of the step's launches (forward, transposed, SDDMM per batch) on one layout,
+    no timing: pass 0 warms up, pass 1 is what an ncu capture selects.  For profiling only."""
     import torch
 
     from sparse_spmm_b200 import build as build_mod
@@ -502,7 +522,17 @@ def run_profile(args) -> None:
 
     build_mod.build()
     torch.cuda.set_device(0)
-    layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
+    relu = False
+    if args.profile_workload == "gpt2-w1":  # GPT-2 c_fc, 3072 x 768 at 90% (magnitude-pruned), fp32, N = 1024
+        layer = wl.magnitude_pruned_layer(3072, 768, 0.90, args.seed, "W1")
+        batches = [1024]
+    elif args.profile_workload == "conv-512x2048-s80":  # 1x1 conv, fp32, N = 6272, X = ReLU(N(0,1))
+        layer = wl.uniform_layer(512, 2048, 0.80, "f32", args.seed, "W")
+        batches = [6272]
+        relu = True
+    else:  # the bench workload
+        layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
+        batches = [int(b) for b in args.batches.split(",")]
 
     def dev_t(a):
         if a.dtype == np.uint16:
@@ -510,9 +540,8 @@ def run_profile(args) -> None:
         return torch.from_numpy(a).cuda()
 
     L = snk.Layout(layer.M, layer.K, dev_t(layer.row), dev_t(layer.col), dev_t(layer.values), num_parts=args.parts)
-    batches = [int(b) for b in args.batches.split(",")]
-    data = {N: (dev_t(wl.activations(layer.K, N, "bf16", args.seed, stream=2)),
-                dev_t(wl.activations(layer.M, N, "bf16", args.seed, stream=3))) for N in batches}
+    data = {N: (dev_t(wl.activations(layer.K, N, layer.dtype, args.seed, stream=2, relu=relu)),
+                dev_t(wl.activations(layer.M, N, layer.dtype, args.seed, stream=3))) for N in batches}
     torch.cuda.synchronize()
     for _ in range(2):
         for N in batches:
@@ -521,7 +550,8 @@ def run_profile(args) -> None:
             L.backward_input(dY)
             L.backward_weight(dY, X)
     torch.cuda.synchronize()
-    print(json.dumps({"profile_passes": 2, "launches_per_pass": 3 * len(batches), "batches": batches}))
+    print(json.dumps({"profile_passes": 2, "launches_per_pass": 3 * len(batches), "batches": batches,
+                      "workload": args.profile_workload}))
 
 
 # ----------------------------------------------------------------------------- sweep over every config
@@ -691,6 +721,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run two untimed passes of the step (for ncu captures) and exit")
+    ap.add_argument("--profile-workload", default="fc", choices=("fc", "gpt2-w1", "conv-512x2048-s80"),
+                    help="workload of --profile: the bench's FC layer, GPT-2 c_fc at N=1024, or a 1x1 conv at N=6272")
     ap.add_argument("--sweep", action="store_true",
                     help="time every config, op and batch (plus dense baselines); JSON lines; exit")
     args = ap.parse_args()

@@ -90,7 +90,8 @@ SNK_API int32_t snk_default_num_parts(int64_t nnz, int32_t sm_count);
 
 /* Bytes of device workspace a layout with these sizes needs (num_parts as passed to
  * snk_build; 0 = the default for the current device, which this call then queries).
- * Returns 0 for invalid sizes.  The size does not change under snk_restructure. */
+ * Returns 0 for invalid sizes.  The size does not change under snk_restructure.  It
+ * includes 4 bytes per nonzero for 16-bit index copies when M, K <= 65536. */
 SNK_API size_t snk_workspace_bytes(int64_t M, int64_t K, int64_t nnz, int32_t num_parts);
 
 /*
@@ -190,6 +191,18 @@ SNK_API snk_status snk_csr_forward_static(int64_t M, int64_t K, int64_t nnz, con
 
 /* Fill *v with the layout's sizes and device pointers.  Returns SNK_ERR_INVALID_ARG for
  * NULL arguments. */
+/*
+ * snk_set_index_bits -- the width of the column / row indices the products read: 32 (the
+ * format as built, the default) or 16.  Index bytes are a cost the essay "Two Lotteries"
+ * names for unstructured formats; when both M and K are <= 65536 the layout also keeps
+ * 16-bit copies of col and csc_row (in the workspace, refreshed by snk_restructure), and
+ * bits = 16 makes the forward, transposed and SDDMM kernels read those instead: 2 bytes
+ * per nonzero less (perm stays 32-bit).  Results are bit-identical either way.  Takes
+ * effect for calls made after it; SNK_ERR_INVALID_ARG for other widths,
+ * SNK_ERR_UNSUPPORTED for 16 when a dimension exceeds 65536.  (A library addition.)
+ */
+SNK_API snk_status snk_set_index_bits(snk_layout* L, int32_t bits);
+
 /*
  * snk_sync_status -- synchronises `stream` and reports whether a product launch on this
  * layout gave up a bounded wait: the TMA-staged kernels for wide operands wait on

@@ -6,9 +6,11 @@
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import os
 import subprocess
 import sys
+import tempfile
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -40,14 +42,24 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every source to an object in parallel (device code split over threads), then
+    link the shared library; objects live in a temporary directory."""
     if not force and not _stale():
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp]
-    if ptxas_verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, f) for f in SOURCES]
-    subprocess.check_call(cmd)
+    with tempfile.TemporaryDirectory(prefix="snk_build_") as objdir:
+        def compile_one(src: str) -> str:
+            obj = os.path.join(objdir, os.path.splitext(src)[0] + ".o")
+            cmd = [_nvcc(), *NVCC_FLAGS, "-split-compile=0", "-I", INCLUDE, "-I", CSRC, "-c",
+                   os.path.join(CSRC, src), "-o", obj]
+            if ptxas_verbose:
+                cmd += ["-Xptxas", "-v"]
+            subprocess.check_call(cmd)
+            return obj
+
+        with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+            objs = list(ex.map(compile_one, SOURCES))
+        subprocess.check_call([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

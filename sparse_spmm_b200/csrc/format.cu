@@ -338,6 +338,12 @@ __global__ void k_part_desc(const int32_t* __restrict__ ptr, int64_t dim, int64_
 
 // ------------------------------------------------------------------------- restructure kernels
 
+// 16-bit copy of an index array whose values are known to be < 65536.
+__global__ void k_narrow(const int32_t* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (uint16_t)in[i];
+}
+
 template <typename W>
 __global__ void k_mag_keys(const W* __restrict__ values, int64_t nnz, uint64_t* __restrict__ keys,
                            uint32_t* __restrict__ vals, uint32_t* err) {
@@ -569,6 +575,13 @@ size_t carve(snk_layout* L, uint8_t* base) {
   L->grown = c.take<uint64_t>(nnz);
   L->vcopy = c.take<uint8_t>(4 * nnz);
   L->scan_tmp = c.take<uint32_t>(ceil_div(L->scap, kScanTile) + ceil_div((int64_t)256 * ceil_div(L->scap, kSortTile), kScanTile) + 64);
+  if (index16_possible(M, K)) {
+    L->col16 = c.take<uint16_t>(nnz);
+    L->csc_row16 = c.take<uint16_t>(nnz);
+  } else {
+    L->col16 = nullptr;
+    L->csc_row16 = nullptr;
+  }
   return c.off;
 }
 
@@ -580,7 +593,7 @@ size_t workspace_bytes(int64_t M, int64_t K, int64_t nnz, int32_t P) {
   L.K = K;
   L.nnz = nnz;
   L.P = P;
-  return carve(&L, nullptr) + 256;
+  return (carve(&L, nullptr) + 256 + 255) / 256 * 256;  // whole 256-byte blocks
 }
 
 snk_status layout_carve(snk_layout* L, void* ws, size_t ws_bytes) {
@@ -609,6 +622,11 @@ snk_status derive_format(snk_layout* L, cudaStream_t s) {
                                                             L->err);
   k_part_desc<<<grid_for(L->P, kThreads), kThreads, 0, s>>>(L->row_ptr, L->M, nnz, L->P, L->part_row, L->desc_f, L->err);
   k_part_desc<<<grid_for(L->P, kThreads), kThreads, 0, s>>>(L->col_ptr, L->K, nnz, L->P, L->part_col, L->desc_t, L->err);
+  SNK_CUDA_TRY(cudaGetLastError());
+  if (L->col16 != nullptr) {
+    k_narrow<<<grid_for(nnz, kThreads), kThreads, 0, s>>>(L->col, L->col16, nnz);
+    k_narrow<<<grid_for(nnz, kThreads), kThreads, 0, s>>>(L->csc_row, L->csc_row16, nnz);
+  }
   SNK_CUDA_TRY(cudaGetLastError());
   SNK_CUDA_TRY(fill_u32(L->cnt_f, (int64_t)kMaxTiles * L->P, 0u, s));
   SNK_CUDA_TRY(fill_u32(L->cnt_b, (int64_t)kMaxTiles * L->P, 0u, s));

@@ -33,6 +33,9 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // the regrowth rounds need (accepted < nnz) + (a batch >= nnz + 4096).
 inline int64_t sort_capacity(int64_t nnz) { return 2 * nnz + 4096; }
 
+// Index arrays fit 16 bits when both dimensions do.
+inline bool index16_possible(int64_t M, int64_t K) { return M <= 65536 && K <= 65536; }
+
 }  // namespace snk
 
 // Host object behind snk_layout.  All pointers are device pointers into the caller's
@@ -49,6 +52,11 @@ struct snk_layout {
   int32_t* col_ptr;
   int32_t* csc_row;
   int32_t* perm;
+  // 16-bit copies of col and csc_row (null unless M, K <= 65536), and the width the
+  // products read (32 unless switched with snk_set_index_bits)
+  uint16_t* col16;
+  uint16_t* csc_row16;
+  int index_bits;
   int32_t* part_nnz;
   int32_t* part_row;
   int32_t* part_nnz_t;

@@ -122,6 +122,7 @@ snk_status snk_build(int64_t M, int64_t K, int64_t nnz, int32_t* row, int32_t* c
   L->sm_count = sms;
   L->row = row;
   L->col = col;
+  L->index_bits = 32;
   snk_status st = snk::layout_carve(L, workspace, ws_bytes);
   if (st == SNK_OK) st = snk::build_format(L, values, elem_bytes(vdt), (cudaStream_t)stream);
   if (st != SNK_OK) {
@@ -178,6 +179,13 @@ snk_status snk_restructure(snk_layout* L, void* values, int64_t drop_count, uint
   return on_device(L->device, [&] {
     return snk::restructure(L, values, drop_count, seed, regrow_value, old_to_new, (cudaStream_t)stream);
   });
+}
+
+snk_status snk_set_index_bits(snk_layout* L, int32_t bits) {
+  if (L == nullptr || (bits != 16 && bits != 32)) return SNK_ERR_INVALID_ARG;
+  if (bits == 16 && (L->col16 == nullptr || L->csc_row16 == nullptr)) return SNK_ERR_UNSUPPORTED;
+  L->index_bits = bits;
+  return SNK_OK;
 }
 
 snk_status snk_sync_status(snk_layout* L, snk_stream stream) {

@@ -230,10 +230,10 @@ __device__ __forceinline__ int64_t search_row(RPF rp, int64_t lo, int64_t hi, in
 
 // ------------------------------------------------------------------------- SpMM (fwd / transposed)
 
-template <typename T>
+template <typename T, typename I>
 struct SpmmArgs {
   const int32_t* ptr;  // [rows + 1] row_ptr (forward) or col_ptr (transposed)
-  const int32_t* idx;  // [nnz] col (forward) or csc_row (transposed)
+  const I* idx;        // [nnz] col (forward) or csc_row (transposed), 32- or 16-bit
   const int32_t* perm; // [nnz] transposed only: sorted-COO index of the j-th CSC entry
   const T* vals;       // [nnz] values in sorted-COO order
   const int4* desc;    // [P] per-CTA work descriptors {a, b, ra, rb}
@@ -265,8 +265,8 @@ constexpr int spmm_batch() {
 template <typename T, int NC>
 constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 32 ? 2 : (NC * (int)sizeof(T) >= 8 ? 4 : 6); }
 
-template <typename T, int NC, int G, bool TRANS>
-__global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A) {
+template <typename T, int NC, int G, bool TRANS, typename I>
+__global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T, I> A) {
   constexpr int NW = kThreads / G;   // workers per CTA
   constexpr int WPW = 32 / G;        // workers per warp
   constexpr int NT = NC * G;         // columns per tile
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
       prefetch_l2(A.desc + part, sizeof(int4));
       prefetch_slice<4>(A.ptr, A.prows, part, A.P);
     } else if (wp == 1) {
-      prefetch_slice<4>(A.idx, A.nnz, part, A.P);
+      prefetch_slice<sizeof(I)>(A.idx, A.nnz, part, A.P);
     } else if (wp == 2) {
       prefetch_slice<sizeof(T)>(A.vals, A.nnz, part, A.P);
     } else if (wp == 3) {
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
   // the worker's piece, as offsets from a
   const int s = (int)(((int64_t)np * w) / NW);
   const int e_end = (int)(((int64_t)np * (w + 1)) / NW);
-  const int32_t* __restrict__ idx = A.idx + a;
+  const I* __restrict__ idx = A.idx + a;
   const int32_t* __restrict__ prm = TRANS ? A.perm + a : nullptr;
   const T* __restrict__ vals = TRANS ? A.vals : A.vals + a;
 
@@ -527,10 +527,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T> A)
 
 // ------------------------------------------------------------------------- SDDMM
 
-template <typename T>
+template <typename T, typename I>
 struct SddmmArgs {
   const int32_t* row_ptr;
-  const int32_t* col;
+  const I* col;      // [nnz], 32- or 16-bit
   const int4* desc;  // [P] per-CTA work descriptors (forward ones)
   const T* X;        // K x N
   const T* dY;       // M x N
@@ -557,8 +557,8 @@ __device__ __forceinline__ float dot_packed(const Packed<T, NC>& x, const Packed
   }
 }
 
-template <typename T, int NC, int G>
-__global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> A) {
+template <typename T, int NC, int G, typename I>
+__global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T, I> A) {
   constexpr int NW = kThreads / G;
   constexpr int NT = NC * G;
   constexpr int UB = sddmm_batch<T, NC>();
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
       prefetch_l2(A.desc + part, sizeof(int4));
       prefetch_slice<4>(A.row_ptr, A.rows + 1, part, P);
     } else if (wp == 1) {
-      prefetch_slice<4>(A.col, A.nnz, part, P);
+      prefetch_slice<sizeof(I)>(A.col, A.nnz, part, P);
     } else if (wp == 2) {
       prefetch_slice<1>(A.X, A.xbytes, part, P);
     } else if (wp == 3) {
@@ -593,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
   const bool staged = np <= kStageCap;
   const int s = (int)(((int64_t)np * w) / NW);
   const int e_end = (int)(((int64_t)np * (w + 1)) / NW);
-  const int32_t* __restrict__ col = A.col + a;
+  const I* __restrict__ col = A.col + a;
   int c[UB];
   auto load_batch = [&](int e0, int nb) {
 #pragma unroll
@@ -689,10 +689,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T> 
 // the shared-memory read of one operand element per FMA.
 constexpr int kWideCols = 128;  // columns per slice (4 per lane)
 
-template <typename T>
+template <typename T, typename I>
 struct WideArgs {
   const int32_t* ptr;   // [rows + 1]
-  const int32_t* idx;   // [nnz], sorted within each row
+  const I* idx;         // [nnz], sorted within each row, 32- or 16-bit
   const int32_t* perm;  // transposed only
   const T* vals;
   const T* B;           // brows x N, leading dimension ldb (16-byte aligned rows)
@@ -789,9 +789,9 @@ __device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
                : "memory");
 }
 
-template <typename T, bool TRANS, int RW>
+template <typename T, bool TRANS, int RW, typename I>
 __global__ void __launch_bounds__(kTmaThreads, 2)
-    k_spmm_tma(const WideArgs<T> A, const __grid_constant__ CUtensorMap tmB) {
+    k_spmm_tma(const WideArgs<T, I> A, const __grid_constant__ CUtensorMap tmB) {
   constexpr int E = (int)sizeof(T);
   constexpr int KC = tma_kc<T, RW>();
   constexpr int ROWB = kWideCols * E;  // bytes of one staged dense row
@@ -919,8 +919,24 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
             float4 x[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) x[u] = load_x(e[u]);
+            if constexpr (E == 2 || RW <= 6) {
+              // two FMA chains of two (odd entries into b01/b23), joined by one packed add
+              float2 b01 = make_float2(0.f, 0.f), b23 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) fma_x(e[u], x[u]);
+              for (int u = 0; u < 4; u += 2) {
+                const float2 v0 = make_float2(__uint_as_float(e[u].x), __uint_as_float(e[u].y));
+                const float2 v1 = make_float2(__uint_as_float(e[u + 1].x), __uint_as_float(e[u + 1].y));
+                a01 = __ffma2_rn(v0, make_float2(x[u].x, x[u].y), a01);
+                a23 = __ffma2_rn(v0, make_float2(x[u].z, x[u].w), a23);
+                b01 = __ffma2_rn(v1, make_float2(x[u + 1].x, x[u + 1].y), b01);
+                b23 = __ffma2_rn(v1, make_float2(x[u + 1].z, x[u + 1].w), b23);
+              }
+              a01 = __fadd2_rn(a01, b01);
+              a23 = __fadd2_rn(a23, b23);
+            } else {  // fp32 with 8 rows per warp: no registers to spare for a second chain
+#pragma unroll
+              for (int u = 0; u < 4; ++u) fma_x(e[u], x[u]);
+            }
           }
           if (t < lim) {  // up to three more: predicated loads first, then the FMAs
             uint4 e[3];
@@ -1088,15 +1104,15 @@ cudaError_t launch_pdl(void (*kern)(const Args), dim3 grid, cudaStream_t s, cons
   return cudaLaunchKernelEx(&cfg, kern, args);
 }
 
-template <typename T, bool TRANS>
-using SpmmKernel = void (*)(const SpmmArgs<T>);
+template <typename T, bool TRANS, typename I>
+using SpmmKernel = void (*)(const SpmmArgs<T, I>);
 
 // Instantiated shapes: 32-byte groups (NC = 16 bf16 / 8 fp32) with G = 1..64/NC lanes,
 // 16-, 8- and 4-byte groups with one lane, and scalars with G = 1..32.
-template <typename T, bool TRANS>
-SpmmKernel<T, TRANS> pick_spmm(int nc, int g) {
+template <typename T, bool TRANS, typename I>
+SpmmKernel<T, TRANS, I> pick_spmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
-  if (nc == NC_ && g == G_) return k_spmm_small<T, NC_, G_, TRANS>;
+  if (nc == NC_ && g == G_) return k_spmm_small<T, NC_, G_, TRANS, I>;
   if constexpr (sizeof(T) == 2) {
     SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4)
     SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
@@ -1109,13 +1125,13 @@ SpmmKernel<T, TRANS> pick_spmm(int nc, int g) {
   return nullptr;
 }
 
-template <typename T>
-using SddmmKernel = void (*)(const SddmmArgs<T>);
+template <typename T, typename I>
+using SddmmKernel = void (*)(const SddmmArgs<T, I>);
 
-template <typename T>
-SddmmKernel<T> pick_sddmm(int nc, int g) {
+template <typename T, typename I>
+SddmmKernel<T, I> pick_sddmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
-  if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_>;
+  if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_, I>;
   if constexpr (sizeof(T) == 2) {
     SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4) SNK_CASE(16, 8) SNK_CASE(16, 16) SNK_CASE(16, 32)
     SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
@@ -1130,8 +1146,8 @@ SddmmKernel<T> pick_sddmm(int nc, int g) {
 
 // The TMA-staged wide kernel; SNK_ERR_UNSUPPORTED (nothing launched) where no tensor map
 // can describe B, so that the caller takes another path.
-template <typename T, bool TRANS, int RW>
-snk_status launch_tma(const WideArgs<T>& A, const T* B, int64_t N, int64_t ldb, int64_t slices, cudaStream_t s) {
+template <typename T, bool TRANS, int RW, typename I>
+snk_status launch_tma(const WideArgs<T, I>& A, const T* B, int64_t N, int64_t ldb, int64_t slices, cudaStream_t s) {
   constexpr int kc = tma_kc<T, RW>();
   CUtensorMap map;
   if (!dense_tensor_map<T>(&map, B, A.brows, N, ldb, kc)) return SNK_ERR_UNSUPPORTED;
@@ -1147,17 +1163,17 @@ snk_status launch_tma(const WideArgs<T>& A, const T* B, int64_t N, int64_t ldb, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, RW>>(smem)));
-  SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, RW>, A, map)));
+  SNK_CUDA_TRY((ensure_dynamic_smem<k_spmm_tma<T, TRANS, RW, I>>(smem)));
+  SNK_CUDA_TRY((cudaLaunchKernelEx(&cfg, k_spmm_tma<T, TRANS, RW, I>, A, map)));
   return SNK_OK;
 }
 
-template <typename T, bool TRANS>
-snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
-                    cudaStream_t s) {
-  WideArgs<T> A;
+template <typename T, bool TRANS, typename I>
+snk_status spmm_tma(const snk_layout* L, const I* idx, const T* values, const T* B, int64_t N, int64_t ldb, T* C,
+                    int64_t ldc, cudaStream_t s) {
+  WideArgs<T, I> A;
   A.ptr = TRANS ? L->col_ptr : L->row_ptr;
-  A.idx = TRANS ? L->csc_row : L->col;
+  A.idx = idx;
   A.perm = TRANS ? L->perm : nullptr;
   A.vals = values;
   A.B = B;
@@ -1183,20 +1199,20 @@ snk_status spmm_tma(const snk_layout* L, const T* values, const T* B, int64_t N,
       best = rw;
     }
   }
-  if (best == 8) return launch_tma<T, TRANS, 8>(A, B, N, ldb, slices, s);
-  if (best == 6) return launch_tma<T, TRANS, 6>(A, B, N, ldb, slices, s);
-  return launch_tma<T, TRANS, 4>(A, B, N, ldb, slices, s);
+  if (best == 8) return launch_tma<T, TRANS, 8, I>(A, B, N, ldb, slices, s);
+  if (best == 6) return launch_tma<T, TRANS, 6, I>(A, B, N, ldb, slices, s);
+  return launch_tma<T, TRANS, 4, I>(A, B, N, ldb, slices, s);
 }
 
-template <typename T, bool TRANS>
-snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t N, int64_t ldb, T* C, int64_t ldc,
-                      cudaStream_t s) {
+template <typename T, bool TRANS, typename I>
+snk_status spmm_typed(const snk_layout* L, const I* idx, const T* values, const T* B, int64_t N, int64_t ldb, T* C,
+                      int64_t ldc, cudaStream_t s) {
   const int elem = (int)sizeof(T);
   const int64_t rows = TRANS ? L->K : L->M;
   // wide operands: the TMA-staged row-block x column-slice kernel where a tensor map can
   // describe B (16-byte aligned base and row stride)
   if (N >= kTmaMinN) {
-    const snk_status st = spmm_tma<T, TRANS>(L, values, B, N, ldb, C, ldc, s);
+    const snk_status st = spmm_tma<T, TRANS, I>(L, idx, values, B, N, ldb, C, ldc, s);
     if (st != SNK_ERR_UNSUPPORTED) return st;
   }
   for (int64_t col0 = 0; col0 < N; col0 += kCarryCols) {
@@ -1213,11 +1229,11 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
     g = std::min(g, 32);
     const int nt = nc * g;
     const int tiles = (ncols + nt - 1) / nt;
-    auto kern = pick_spmm<T, TRANS>(nc, g);
+    auto kern = pick_spmm<T, TRANS, I>(nc, g);
     if (kern == nullptr || tiles > kMaxTiles) return SNK_ERR_UNSUPPORTED;
-    SpmmArgs<T> A;
+    SpmmArgs<T, I> A;
     A.ptr = TRANS ? L->col_ptr : L->row_ptr;
-    A.idx = TRANS ? L->csc_row : L->col;
+    A.idx = idx;
     A.perm = TRANS ? L->perm : nullptr;
     A.vals = values;
     A.desc = TRANS ? L->desc_t : L->desc_f;
@@ -1241,23 +1257,23 @@ snk_status spmm_typed(const snk_layout* L, const T* values, const T* B, int64_t 
   return SNK_OK;
 }
 
-template <typename T>
-snk_status sddmm_typed(const snk_layout* L, const T* dY, int64_t lddy, const T* X, int64_t ldx, int64_t N, T* dW,
-                       cudaStream_t s) {
+template <typename T, typename I>
+snk_status sddmm_typed(const snk_layout* L, const I* col, const T* dY, int64_t lddy, const T* X, int64_t ldx,
+                       int64_t N, T* dW, cudaStream_t s) {
   const int elem = (int)sizeof(T);
   const int ncap = (int)std::min<int64_t>(N, 1 << 20);
   int nc = pick_nc(std::max(ncap, 1), elem, X, ldx, dY, lddy);
   int g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>((N + nc - 1) / nc, 64)));
-  auto kern = pick_sddmm<T>(nc, g);
+  auto kern = pick_sddmm<T, I>(nc, g);
   if (kern == nullptr) {
     nc = 1;
     g = (int)std::min<int64_t>(32, pow2ceil((int)std::max<int64_t>(1, std::min<int64_t>(N, 64))));
-    kern = pick_sddmm<T>(nc, g);
+    kern = pick_sddmm<T, I>(nc, g);
   }
   if (kern == nullptr) return SNK_ERR_UNSUPPORTED;
-  SddmmArgs<T> A;
+  SddmmArgs<T, I> A;
   A.row_ptr = L->row_ptr;
-  A.col = L->col;
+  A.col = col;
   A.desc = L->desc_f;
   A.X = X;
   A.dY = dY;
@@ -1289,26 +1305,48 @@ snk_status launch_zero_rows(void* C, int64_t rows, int64_t N, int64_t ldc, int e
   return SNK_OK;
 }
 
+namespace {
+
+// Entry points by value type and index width: the 16-bit copies of the index arrays are
+// used when the layout is switched to them (and holds them).
+template <typename T>
+snk_status spmm_by_index(const snk_layout* L, bool transpose, const T* values, const T* B, int64_t N, int64_t ldb,
+                         T* C, int64_t ldc, cudaStream_t s) {
+  if (L->index_bits == 16 && L->col16 != nullptr && L->csc_row16 != nullptr) {
+    return transpose ? spmm_typed<T, true, uint16_t>(L, L->csc_row16, values, B, N, ldb, C, ldc, s)
+                     : spmm_typed<T, false, uint16_t>(L, L->col16, values, B, N, ldb, C, ldc, s);
+  }
+  return transpose ? spmm_typed<T, true, int32_t>(L, L->csc_row, values, B, N, ldb, C, ldc, s)
+                   : spmm_typed<T, false, int32_t>(L, L->col, values, B, N, ldb, C, ldc, s);
+}
+
+template <typename T>
+snk_status sddmm_by_index(const snk_layout* L, const T* dY, int64_t lddy, const T* X, int64_t ldx, int64_t N, T* dW,
+                          cudaStream_t s) {
+  if (L->index_bits == 16 && L->col16 != nullptr)
+    return sddmm_typed<T, uint16_t>(L, L->col16, dY, lddy, X, ldx, N, dW, s);
+  return sddmm_typed<T, int32_t>(L, L->col, dY, lddy, X, ldx, N, dW, s);
+}
+
+}  // namespace
+
 snk_status launch_spmm(const snk_layout* L, bool transpose, const void* values, const void* B, int64_t N, int64_t ldb,
                        void* C, int64_t ldc, cudaStream_t s) {
   const int64_t rows = transpose ? L->K : L->M;
   if (L->nnz == 0) return launch_zero_rows(C, rows, N, ldc, L->dtype == SNK_F32 ? 4 : 2, s);
-  if (L->dtype == SNK_F32) {
-    return transpose ? spmm_typed<float, true>(L, (const float*)values, (const float*)B, N, ldb, (float*)C, ldc, s)
-                     : spmm_typed<float, false>(L, (const float*)values, (const float*)B, N, ldb, (float*)C, ldc, s);
-  }
+  if (L->dtype == SNK_F32)
+    return spmm_by_index<float>(L, transpose, (const float*)values, (const float*)B, N, ldb, (float*)C, ldc, s);
   using bf = __nv_bfloat16;
-  return transpose ? spmm_typed<bf, true>(L, (const bf*)values, (const bf*)B, N, ldb, (bf*)C, ldc, s)
-                   : spmm_typed<bf, false>(L, (const bf*)values, (const bf*)B, N, ldb, (bf*)C, ldc, s);
+  return spmm_by_index<bf>(L, transpose, (const bf*)values, (const bf*)B, N, ldb, (bf*)C, ldc, s);
 }
 
 snk_status launch_sddmm(const snk_layout* L, const void* dY, int64_t lddy, const void* X, int64_t ldx, int64_t N,
                         void* dW, cudaStream_t s) {
   if (L->nnz == 0) return SNK_OK;
   if (L->dtype == SNK_F32)
-    return sddmm_typed<float>(L, (const float*)dY, lddy, (const float*)X, ldx, N, (float*)dW, s);
+    return sddmm_by_index<float>(L, (const float*)dY, lddy, (const float*)X, ldx, N, (float*)dW, s);
   using bf = __nv_bfloat16;
-  return sddmm_typed<bf>(L, (const bf*)dY, lddy, (const bf*)X, ldx, N, (bf*)dW, s);
+  return sddmm_by_index<bf>(L, (const bf*)dY, lddy, (const bf*)X, ldx, N, (bf*)dW, s);
 }
 
 }  // namespace snk

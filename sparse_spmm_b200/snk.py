@@ -179,6 +179,14 @@ def snk_csr_forward_static(M, K, row_ptr, col, values, X, Y, num_parts=0, stream
               _ld(X), _ptr(Y), _ld(Y), num_parts, _stream(stream)), "snk_csr_forward_static")
 
 
+def snk_set_index_bits(handle, bits):
+    """Read 16- or 32-bit indices in the products (16 needs M, K <= 65536)."""
+    lib = load_library()
+    lib.snk_set_index_bits.restype = ctypes.c_int
+    lib.snk_set_index_bits.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    _check(lib.snk_set_index_bits(handle, bits), "snk_set_index_bits")
+
+
 def snk_sync_status(handle, stream=None):
     """Synchronise and raise SnkError(SNK_ERR_TIMEOUT) if a product launch gave up a wait."""
     lib = load_library()
@@ -273,6 +281,10 @@ class Layout:
         snk_restructure(self.handle, self.values, drop_count, seed, regrow_value, o2n, stream)
         return o2n
 
+    def set_index_bits(self, bits: int):
+        """Make the products read 16- or 32-bit indices (results are bit-identical)."""
+        snk_set_index_bits(self.handle, bits)
+
     def sync_status(self, stream=None):
         """Synchronise; raise if a product launch on this layout gave up a bounded wait."""
         snk_sync_status(self.handle, stream)
@@ -282,11 +294,11 @@ class Layout:
         """Device arrays of the layout as int32 tensors (views of the workspace)."""
         v = snk_layout_info(self.handle)
         base = self.workspace.data_ptr()
-        ws32 = self.workspace.view(torch.int32) if self.workspace.numel() % 4 == 0 else None
+        ws32 = self.workspace[: self.workspace.numel() // 4 * 4].view(torch.int32)
 
         def sl(ptr, n):
             off = ptr - base
-            assert off % 4 == 0 and ws32 is not None
+            assert off % 4 == 0
             return ws32[off // 4: off // 4 + n]
 
         P = int(v.num_parts)
