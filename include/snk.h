@@ -192,6 +192,18 @@ SNK_API snk_status snk_csr_forward_static(int64_t M, int64_t K, int64_t nnz, con
 /* Fill *v with the layout's sizes and device pointers.  Returns SNK_ERR_INVALID_ARG for
  * NULL arguments. */
 /*
+ * snk_remap_entries -- carries per-entry state (optimizer moments, masks, ...) across a
+ * snk_restructure: dst[old_to_new[e]] = src[e] for every e with old_to_new[e] >= 0, and
+ * every other dst entry (the regrown connections) is set to zero.  old_to_new: the int32
+ * [nnz] map snk_restructure wrote; src, dst: device [nnz] arrays of elem_bytes (2 or 4)
+ * each, not aliased.  Asynchronous on `stream` (on the current device); SNK_ERR_INVALID_ARG
+ * for bad sizes, null or aliased pointers.  (A library addition: the training loop of
+ * dynamic sparse training needs it; the pages name the use, not the call.)
+ */
+SNK_API snk_status snk_remap_entries(const int32_t* old_to_new, int64_t nnz, const void* src, void* dst,
+                                     int32_t elem_bytes, snk_stream stream);
+
+/*
  * snk_set_index_bits -- the width of the column / row indices the products read: 32 (the
  * format as built, the default) or 16.  Index bytes are a cost the essay "Two Lotteries"
  * names for unstructured formats; when both M and K are <= 65536 the layout also keeps

@@ -344,6 +344,16 @@ __global__ void k_narrow(const int32_t* __restrict__ in, uint16_t* __restrict__ 
     out[i] = (uint16_t)in[i];
 }
 
+// dst[old_to_new[e]] = src[e] for the surviving entries of a restructure (dst zeroed first).
+template <typename W>
+__global__ void k_remap_scatter(const int32_t* __restrict__ old_to_new, int64_t nnz, const W* __restrict__ src,
+                                W* __restrict__ dst) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nnz; e += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t t = old_to_new[e];
+    if (t >= 0 && t < nnz) dst[t] = src[e];
+  }
+}
+
 template <typename W>
 __global__ void k_mag_keys(const W* __restrict__ values, int64_t nnz, uint64_t* __restrict__ keys,
                            uint32_t* __restrict__ vals, uint32_t* err) {
@@ -758,6 +768,20 @@ snk_status restructure(snk_layout* L, void* values, int64_t k, uint64_t seed, fl
   SNK_TRY(derive_format(L, s));
   SNK_TRY(read_err(L, s, &e));
   return status_from_err(e);
+}
+
+snk_status remap_entries(const int32_t* old_to_new, int64_t nnz, const void* src, void* dst, int elem_bytes,
+                         cudaStream_t s) {
+  if (nnz == 0) return SNK_OK;
+  SNK_CUDA_TRY(cudaMemsetAsync(dst, 0, (size_t)nnz * (size_t)elem_bytes, s));
+  if (elem_bytes == 4)
+    k_remap_scatter<uint32_t><<<grid_for(nnz, kThreads), kThreads, 0, s>>>(old_to_new, nnz, (const uint32_t*)src,
+                                                                           (uint32_t*)dst);
+  else
+    k_remap_scatter<uint16_t><<<grid_for(nnz, kThreads), kThreads, 0, s>>>(old_to_new, nnz, (const uint16_t*)src,
+                                                                           (uint16_t*)dst);
+  SNK_CUDA_TRY(cudaGetLastError());
+  return SNK_OK;
 }
 
 }  // namespace snk

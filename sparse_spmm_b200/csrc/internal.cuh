@@ -105,6 +105,8 @@ snk_status launch_spmm(const snk_layout* L, bool transpose, const void* values, 
 snk_status launch_sddmm(const snk_layout* L, const void* dY, int64_t lddy, const void* X, int64_t ldx,
                         int64_t N, void* dW, cudaStream_t s);
 snk_status launch_zero_rows(void* C, int64_t rows, int64_t N, int64_t ldc, int elem_bytes, cudaStream_t s);
+snk_status remap_entries(const int32_t* old_to_new, int64_t nnz, const void* src, void* dst, int elem_bytes,
+                         cudaStream_t s);
 
 }  // namespace snk
 

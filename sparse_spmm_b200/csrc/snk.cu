@@ -181,6 +181,13 @@ snk_status snk_restructure(snk_layout* L, void* values, int64_t drop_count, uint
   });
 }
 
+snk_status snk_remap_entries(const int32_t* old_to_new, int64_t nnz, const void* src, void* dst, int32_t elem_bytes,
+                             snk_stream stream) {
+  if (nnz < 0 || (elem_bytes != 2 && elem_bytes != 4)) return SNK_ERR_INVALID_ARG;
+  if (nnz > 0 && (old_to_new == nullptr || src == nullptr || dst == nullptr || src == dst)) return SNK_ERR_INVALID_ARG;
+  return snk::remap_entries(old_to_new, nnz, src, dst, elem_bytes, (cudaStream_t)stream);
+}
+
 snk_status snk_set_index_bits(snk_layout* L, int32_t bits) {
   if (L == nullptr || (bits != 16 && bits != 32)) return SNK_ERR_INVALID_ARG;
   if (bits == 16 && (L->col16 == nullptr || L->csc_row16 == nullptr)) return SNK_ERR_UNSUPPORTED;

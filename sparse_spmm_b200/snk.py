@@ -179,6 +179,17 @@ def snk_csr_forward_static(M, K, row_ptr, col, values, X, Y, num_parts=0, stream
               _ld(X), _ptr(Y), _ld(Y), num_parts, _stream(stream)), "snk_csr_forward_static")
 
 
+def snk_remap_entries(old_to_new, src, dst, stream=None):
+    """dst[old_to_new[e]] = src[e] for surviving entries, 0 elsewhere (state across a restructure)."""
+    lib = load_library()
+    lib.snk_remap_entries.restype = ctypes.c_int
+    lib.snk_remap_entries.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_int32, ctypes.c_void_p]
+    _check(lib.snk_remap_entries(_ptr(old_to_new), src.numel(), _ptr(src), _ptr(dst), src.element_size(),
+                                 _stream(stream)), "snk_remap_entries")
+    return dst
+
+
 def snk_set_index_bits(handle, bits):
     """Read 16- or 32-bit indices in the products (16 needs M, K <= 65536)."""
     lib = load_library()
