@@ -83,7 +83,7 @@ def test_short_dst_run():
         loss = ((Y - T) ** 2).mean()
         loss.backward()
         opt.step()
-        losses.append(float(loss))
+        losses.append(float(loss.detach()))
     assert (W1.nnz, W2.nnz) == nnz0
     assert np.all(np.isfinite(losses))
     assert losses[-1] < 0.75 * losses[0], losses[::10]
