@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.cuh"
@@ -701,6 +702,7 @@ struct WideArgs {
   int64_t rows, brows;
   int N;
   uint32_t* err;        // status word (may be null): ERRBIT_TIMEOUT if a pipeline wait gave up
+  uint32_t extra_tx;    // 0; a test sets it (environment) so that no chunk ever completes
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -838,7 +840,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
         }
         if (s_abort) break;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(full0 + 8 * st, (uint32_t)CHUNK);
+        mbar_expect_tx(full0 + 8 * st, (uint32_t)CHUNK + A.extra_tx);
         tma_load_2d(xs + st * CHUNK, &tmB, n0, (int)(issued * KC), full0 + 8 * st);
       }
     }
@@ -1144,6 +1146,18 @@ SddmmKernel<T, I> pick_sddmm(int nc, int g) {
   return nullptr;
 }
 
+// Test hook for the bounded waits: SNK_TEST_TMA_EXTRA_TX=<bytes> in the environment makes
+// every chunk expect that many bytes more than its copy delivers, so no "full" barrier ever
+// completes and every wait of the kernel runs out (about a second each); the kernel then
+// reports ERRBIT_TIMEOUT and returns.  Nothing faults and no copy is left in flight.  Unset
+// (the normal case) it is 0.
+uint32_t tma_test_extra_tx() {
+  const char* e = std::getenv("SNK_TEST_TMA_EXTRA_TX");
+  if (e == nullptr) return 0u;
+  const long v = std::strtol(e, nullptr, 10);
+  return (v > 0 && v <= 4096) ? (uint32_t)v : 0u;
+}
+
 // The TMA-staged wide kernel; SNK_ERR_UNSUPPORTED (nothing launched) where no tensor map
 // can describe B, so that the caller takes another path.
 template <typename T, bool TRANS, int RW, typename I>
@@ -1184,6 +1198,7 @@ snk_status spmm_tma(const snk_layout* L, const I* idx, const T* values, const T*
   A.brows = TRANS ? L->M : L->K;
   A.N = (int)N;
   A.err = L->err;
+  A.extra_tx = tma_test_extra_tx();
   const int64_t slices = (N + kWideCols - 1) / kWideCols;
   if (N >= ((int64_t)1 << 31) || slices > 65535) return SNK_ERR_UNSUPPORTED;
   // rows per consumer warp: the choice among 8, 6 and 4 with the shortest estimated
