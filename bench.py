@@ -630,8 +630,9 @@ def fp32_fma_peak(sm_count: int) -> dict:
 def run_sweep(args) -> None:
     """Every config, op and batch of the workload list: L2-cold per-op CUDA graphs, achieved
     GB/s and GFLOP/s under the byte model, fractions of the measured HBM and fp32 FMA peaks,
-    and (forward) the dense and dense+mask products of the same W on the same GPU
-    (torch.matmul, i.e. cuBLAS), as the pages' ratio style.  One JSON line per measurement."""
+    a single launch after an L2 flush, and (forward) the dense and dense+mask products of the
+    same W on the same GPU (torch.matmul, i.e. cuBLAS), as the pages' ratio style.  One JSON
+    line per measurement."""
     import torch
 
     from sparse_spmm_b200 import build as build_mod
@@ -654,6 +655,7 @@ def run_sweep(args) -> None:
     f32["clocks"] = clk.summary()
     print(json.dumps({"sweep": "fp32_fma_peak", **f32}), flush=True)
 
+    flush = torch.empty(3 * l2 // 4, dtype=torch.float32, device="cuda")
     works = [wl.tiny_fc(), wl.fc_4096(), wl.gpt2_mlp(), wl.llama_mlp()]
     works += [wl.conv1x1(M, K, sp) for (M, K) in wl.CONV_SHAPES for sp in wl.CONV_SPARSITIES]
     opname = {"forward": "forward", "backward_input": "backward_input", "backward_weight": "backward_weight"}
@@ -683,10 +685,21 @@ def run_sweep(args) -> None:
                     else:
                         fns = [lambda i=i: copies[i].backward_weight(dY[i], X[i], dW=dW[i]) for i in range(R)]
                     us = _graph_time_us(fns, reps=3 if N >= 1024 else 10)
+                    # one launch right after an L2 flush (a 3 x L2 buffer written), best of 3
+                    single = float("inf")
+                    for _ in range(3):
+                        flush.fill_(1.0)
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        fns[0]()
+                        e1.record()
+                        e1.synchronize()
+                        single = min(single, e0.elapsed_time(e1) * 1e3)
                     b = op_bytes(opname[op], M, K, nnz, N, s)
                     fl = op_flops(nnz, N)
                     rec = {"sweep": work.name, "layer": layer.name, "M": M, "K": K, "nnz": nnz, "op": op, "N": N,
-                           "us": round(us, 2), "gbs": round(b / us / 1e3, 1),
+                           "us": round(us, 2), "single_launch_us": round(single, 2), "gbs": round(b / us / 1e3, 1),
                            "frac_hbm": round(b / us / 1e3 / pk["hbm_gbs"], 4),
                            "gflops": round(fl / us / 1e3, 1), "frac_fp32": round(fl / us / 1e6 / f32["tflops"], 4),
                            "bound": "alu" if fl / (f32["tflops"] * 1e12) > b / (pk["hbm_gbs"] * 1e9) else "hbm"}
