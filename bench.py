@@ -281,12 +281,16 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
                 del g
         return res
 
+    torch.cuda.nvtx.range_push("per-op graphs, int32 indices")
     per_op = time_ops(4)
+    torch.cuda.nvtx.range_pop()
     # the same ops reading 16-bit column / row indices (bit-identical results), with their
     # own byte model; the step above and the headline use the int32 format
     for c in copies:
         c["L"].set_index_bits(16)
+    torch.cuda.nvtx.range_push("per-op graphs, 16-bit indices")
     per_op16 = time_ops(2)
+    torch.cuda.nvtx.range_pop()
     for c in copies:
         c["L"].set_index_bits(32)
     us32 = sum(v["us"] for v in per_op.values())
@@ -306,12 +310,14 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
     e1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("timed steps")
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(args.steps):
                 graphs[i % R].replay()
             e1.record(stream)
         e1.synchronize()
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -369,10 +375,12 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
         e2e_step(copies[i % R])
     torch.cuda.synchronize()
     barrier(world)
+    torch.cuda.nvtx.range_push("e2e steps")
     e0.record(h2d_s)
     for i in range(e2e_steps):
         e2e_step(copies[i % R])
     e1.record(d2h_s)
+    torch.cuda.nvtx.range_pop()
     e1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps

@@ -323,6 +323,27 @@ class Layout:
         }
 
 
+def save_layout(L: Layout, path) -> None:
+    """Checkpoint a layout: its sizes, part count and sorted COO (row, col, value bits).  The
+    derived arrays are state of the build, so a load rebuilds them (byte-identical)."""
+    import numpy as np
+    torch.cuda.synchronize(L.row.device)
+    vbits = L.values.view(torch.int16) if L.values.dtype == torch.bfloat16 else L.values.view(torch.int32)
+    np.savez(path, M=L.M, K=L.K, num_parts=L.num_parts,
+             dtype="bf16" if L.values.dtype == torch.bfloat16 else "f32",
+             row=L.row.cpu().numpy(), col=L.col.cpu().numpy(), value_bits=vbits.cpu().numpy())
+
+
+def load_layout(path, device="cuda") -> Layout:
+    """Rebuild a layout saved by save_layout on `device`."""
+    import numpy as np
+    z = np.load(path)
+    bits_t = torch.from_numpy(z["value_bits"]).to(device)
+    values = bits_t.view(torch.bfloat16) if str(z["dtype"]) == "bf16" else bits_t.view(torch.float32)
+    return Layout(int(z["M"]), int(z["K"]), torch.from_numpy(z["row"]).to(device),
+                  torch.from_numpy(z["col"]).to(device), values.contiguous(), num_parts=int(z["num_parts"]))
+
+
 class SparseLinearFunction(torch.autograd.Function):
     """Y = W X with W held by a Layout; backward returns dX = W^T dY and dW (per entry).
 
