@@ -732,15 +732,17 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
 // depth apart.  Every wait is bounded (about a second by the global timer); one that gives
 // up sets ERRBIT_TIMEOUT in the status word, all roles stop, the producer lets its issued
 // copies land (again bounded), and the CTA returns.
-constexpr int kTmaStages = 3;
+constexpr int kTmaStages = 2;
 constexpr int kTmaMinN = 256;     // narrower operands take 64-column passes of the small kernel
 constexpr int kTmaConsumers = 8;  // compute warps; one more warp produces
 constexpr int kTmaThreads = 32 * (kTmaConsumers + 1);
 
-// Dense rows per staged chunk: as many (up to 64) as let two CTAs -- ring plus entry
-// buffers -- share one SM's shared memory.
+// Dense rows per staged chunk: as many as let two CTAs -- ring plus entry buffers -- share
+// one SM's shared memory.  Two stages of long chunks measured faster than three of short
+// ones: the per-(row, chunk) costs (ballot, tail) fall with more entries per chunk, and one
+// chunk in flight covers the copy latency.
 template <typename T, int RW>
-constexpr int tma_kc() { return sizeof(T) == 2 ? 64 : (RW >= 8 ? 48 : (RW >= 6 ? 56 : 64)); }
+constexpr int tma_kc() { return sizeof(T) == 2 ? 128 : (RW >= 8 ? 72 : (RW >= 6 ? 84 : 96)); }
 
 __device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
