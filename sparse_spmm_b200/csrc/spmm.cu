@@ -725,7 +725,7 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
 // counted on a "full" mbarrier per stage.  Eight consumer warps each own RW rows of the
 // row block and walk every chunk: per row, the entries that fall into the chunk are a
 // prefix of the row's current 32-entry batch (found by a ballot), each broadcast from
-// shared memory as {v, v, dense-row byte offset} so that a lane needs one 16-byte read, one
+// shared memory as {v, dense-row byte offset} so that a lane needs one 8-byte read, one
 // dense-row read and two packed FMAs per entry.  A consumer warp releases a stage by
 // arriving on its "empty" mbarrier; the producer refills a stage once all eight have
 // released it, so no CTA-wide barrier sits in the loop and warps drift up to the ring
@@ -737,12 +737,23 @@ constexpr int kTmaMinN = 256;     // narrower operands take 64-column passes of 
 constexpr int kTmaConsumers = 8;  // compute warps; one more warp produces
 constexpr int kTmaThreads = 32 * (kTmaConsumers + 1);
 
-// Dense rows per staged chunk: as many as let two CTAs -- ring plus entry buffers -- share
-// one SM's shared memory.  Two stages of long chunks measured faster than three of short
-// ones: the per-(row, chunk) costs (ballot, tail) fall with more entries per chunk, and one
-// chunk in flight covers the copy latency.
+// Bytes of one broadcast entry in shared memory: 8 = {v, offset}, or 16 = {v, v, offset, 0}
+// (the value pair ready for the packed FMA, no move per entry).  8 measured 10-20% faster:
+// the space it frees goes to longer chunks.
+constexpr int kTmaEntryBytes = 8;
+
+// Dense rows per staged chunk: the most (a multiple of 8, at most 256) that let two CTAs --
+// ring, entry buffers, barriers and the 1 KB the runtime reserves per CTA -- share one SM's
+// 228 KB.  Two stages of long chunks measured faster than three of short ones: the
+// per-(row, chunk) costs (ballot, tail) fall with more entries per chunk, and one chunk in
+// flight covers the copy latency.
 template <typename T, int RW>
-constexpr int tma_kc() { return sizeof(T) == 2 ? 128 : (RW >= 8 ? 72 : (RW >= 6 ? 84 : 96)); }
+constexpr int tma_kc() {
+  constexpr int kPerCta = 233472 / 2 - 1024;  // bytes of shared memory for each of two CTAs
+  constexpr int stat = 8 * RW * 32 * kTmaEntryBytes + 8 * RW * 8 + 64;
+  constexpr int kc = (kPerCta - stat - 128) / (2 * 128 * (int)sizeof(T)) / 8 * 8;
+  return kc > 256 ? 256 : kc;
+}
 
 __device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
@@ -801,7 +812,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
   constexpr int ROWB = kWideCols * E;  // bytes of one staged dense row
   constexpr int CHUNK = KC * ROWB;     // bytes of one staged chunk (the TMA box)
   extern __shared__ __align__(16) unsigned char s_tx[];  // [kTmaStages][CHUNK] from a 128-byte boundary
-  __shared__ __align__(16) uint4 s_ent[kTmaConsumers][RW][32];  // {v, v, dense-row byte offset, 0}
+  __shared__ __align__(16) unsigned char s_ent[kTmaConsumers][RW][32][kTmaEntryBytes];
   __shared__ int2 s_span[kTmaConsumers][RW];  // per row: {first entry of the current batch, row end}
   __shared__ __align__(8) uint64_t s_full[kTmaStages];
   __shared__ __align__(8) uint64_t s_empty[kTmaStages];
@@ -866,7 +877,11 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
         if (TRANS) asm volatile("prefetch.global.L1 [%0];" ::"l"(A.perm + j));
       }
     };
-    const uint32_t ent0 = smem_addr(&s_ent[wp][0][0]);
+    const uint32_t ent0 = smem_addr(&s_ent[wp][0][0][0]);
+    auto ent_store = [&](uint32_t a, const uint4& e) {
+      if constexpr (kTmaEntryBytes == 16) sts128u(a, e);
+      else asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(e.x), "r"(e.z) : "memory");
+    };
     static_for<0, RW>([&](auto ic) {
       constexpr int i = decltype(ic)::value;
       acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
@@ -878,7 +893,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
       k[i] = 0;
       uint4 ent;
       load_entry(rbeg, rend, cl[i], ent);
-      sts128u(ent0 + (i * 32 + lane) * 16, ent);
+      ent_store(ent0 + (i * 32 + lane) * kTmaEntryBytes, ent);
       prefetch_next(rbeg, rend);
     });
     __syncwarp();
@@ -898,7 +913,15 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
       const int cbound = (int)mn64(kc + KC, A.brows);  // columns below it are staged
       static_for<0, RW>([&](auto ic) {
         constexpr int i = decltype(ic)::value;
-        const uint32_t eb = ent0 + i * 32 * 16;
+        const uint32_t eb = ent0 + i * 32 * kTmaEntryBytes;
+        auto ent_load = [&](int tt) -> uint4 {
+          if constexpr (kTmaEntryBytes == 16) {
+            return lds128u(eb + tt * 16);
+          } else {
+            const uint2 w = lds64(eb + tt * 8);
+            return make_uint4(w.x, w.x, w.y, 0u);
+          }
+        };
         float2 a01 = acc[i][0], a23 = acc[i][1];
         auto fma_x = [&](const uint4& e, const float4& x) {
           const float2 vv = make_float2(__uint_as_float(e.x), __uint_as_float(e.y));
@@ -919,7 +942,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
           for (; t + 4 <= lim; t += 4) {
             uint4 e[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) e[u] = lds128u(eb + (t + u) * 16);
+            for (int u = 0; u < 4; ++u) e[u] = ent_load(t + u);
             float4 x[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) x[u] = load_x(e[u]);
@@ -952,7 +975,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
             }
 #pragma unroll
             for (int u = 0; u < 3; ++u)
-              if (t + u < lim) e[u] = lds128u(eb + (t + u) * 16);
+              if (t + u < lim) e[u] = ent_load(t + u);
 #pragma unroll
             for (int u = 0; u < 3; ++u)
               if (t + u < lim) x[u] = load_x(e[u]);
@@ -968,7 +991,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
           uint4 ent;
           load_entry(nb, sp.y, cl[i], ent);
           __syncwarp();
-          sts128u(eb + lane * 16, ent);
+          ent_store(eb + lane * kTmaEntryBytes, ent);
           if (lane == 0) s_span[wp][i].x = nb;
           __syncwarp();
           k[i] = 0;
