@@ -794,12 +794,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(map), "r"(x), "r"(y), "r"(mbar)
       : "memory");
 }
-__device__ __forceinline__ uint4 lds128u(uint32_t a) {
+[[maybe_unused]] __device__ __forceinline__ uint4 lds128u(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
-__device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
+[[maybe_unused]] __device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
