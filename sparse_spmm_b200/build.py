@@ -42,16 +42,16 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile every source to an object in parallel (device code split over threads), then
-    link the shared library; objects live in a temporary directory."""
+    """Compile every source to an object in parallel, then link the shared library; objects
+    live in a temporary directory."""
     if not force and not _stale():
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
     with tempfile.TemporaryDirectory(prefix="snk_build_") as objdir:
         def compile_one(src: str) -> str:
             obj = os.path.join(objdir, os.path.splitext(src)[0] + ".o")
-            cmd = [_nvcc(), *NVCC_FLAGS, "-split-compile=0", "-I", INCLUDE, "-I", CSRC, "-c",
-                   os.path.join(CSRC, src), "-o", obj]
+            # (no -split-compile: splitting a translation unit's optimisation measured slower code)
+            cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj]
             if ptxas_verbose:
                 cmd += ["-Xptxas", "-v"]
             subprocess.check_call(cmd)

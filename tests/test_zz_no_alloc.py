@@ -56,7 +56,7 @@ def _check_against_forward(layer, Ns, num_parts=0):
 
 def test_static_forward_matches_forward_twice():
     layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", 0, "W")
-    _check_against_forward(layer, (8, 32))
+    _check_against_forward(layer, (8, 32, 300))
 
 
 def test_static_forward_long_rows_and_ragged_batch():
