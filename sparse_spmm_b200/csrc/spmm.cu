@@ -263,8 +263,12 @@ template <typename T, int NC, bool TRANS = false>
 constexpr int spmm_batch() {
   return NC * (int)sizeof(T) >= 32 ? 3 : (NC * (int)sizeof(T) >= 16 ? (perm_ahead<T, NC, TRANS>() ? 5 : 6) : 8);
 }
-template <typename T, int NC>
-constexpr int sddmm_batch() { return NC * (int)sizeof(T) >= 32 ? 2 : (NC * (int)sizeof(T) >= 8 ? 4 : 6); }
+// SDDMM entries in flight per worker.  DEEP (wide operands, several column passes per entry)
+// measured best with more entries in flight, short operands with fewer (registers).
+template <typename T, int NC, bool DEEP = false>
+constexpr int sddmm_batch() {
+  return NC * (int)sizeof(T) >= 32 ? (DEEP ? 4 : 3) : (NC * (int)sizeof(T) >= 8 ? 4 : 6);
+}
 
 template <typename T, int NC, int G, bool TRANS, typename I>
 __global__ void __launch_bounds__(kThreads, 3) k_spmm_small(const SpmmArgs<T, I> A) {
@@ -558,11 +562,11 @@ __device__ __forceinline__ float dot_packed(const Packed<T, NC>& x, const Packed
   }
 }
 
-template <typename T, int NC, int G, typename I>
+template <typename T, int NC, int G, typename I, bool DEEP>
 __global__ void __launch_bounds__(kThreads, 3) k_sddmm_small(const SddmmArgs<T, I> A) {
   constexpr int NW = kThreads / G;
   constexpr int NT = NC * G;
-  constexpr int UB = sddmm_batch<T, NC>();
+  constexpr int UB = sddmm_batch<T, NC, DEEP>();
   __shared__ int32_t s_rp[kRowCap];
   __shared__ float s_dw[kStageCap];
 
@@ -1156,9 +1160,10 @@ template <typename T, typename I>
 using SddmmKernel = void (*)(const SddmmArgs<T, I>);
 
 template <typename T, typename I>
-SddmmKernel<T, I> pick_sddmm(int nc, int g) {
+SddmmKernel<T, I> pick_sddmm(int nc, int g, bool deep) {
+  if (deep && g == 32 && nc * (int)sizeof(T) == 32) return k_sddmm_small<T, 32 / (int)sizeof(T), 32, I, true>;
 #define SNK_CASE(NC_, G_) \
-  if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_, I>;
+  if (nc == NC_ && g == G_) return k_sddmm_small<T, NC_, G_, I, false>;
   if constexpr (sizeof(T) == 2) {
     SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4) SNK_CASE(16, 8) SNK_CASE(16, 16) SNK_CASE(16, 32)
     SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
@@ -1304,11 +1309,11 @@ snk_status sddmm_typed(const snk_layout* L, const I* col, const T* dY, int64_t l
   const int ncap = (int)std::min<int64_t>(N, 1 << 20);
   int nc = pick_nc(std::max(ncap, 1), elem, X, ldx, dY, lddy);
   int g = (int)std::min<int64_t>(32, pow2ceil((int)std::min<int64_t>((N + nc - 1) / nc, 64)));
-  auto kern = pick_sddmm<T, I>(nc, g);
+  auto kern = pick_sddmm<T, I>(nc, g, N >= 256);
   if (kern == nullptr) {
     nc = 1;
     g = (int)std::min<int64_t>(32, pow2ceil((int)std::max<int64_t>(1, std::min<int64_t>(N, 64))));
-    kern = pick_sddmm<T, I>(nc, g);
+    kern = pick_sddmm<T, I>(nc, g, false);
   }
   if (kern == nullptr) return SNK_ERR_UNSUPPORTED;
   SddmmArgs<T, I> A;
