@@ -120,6 +120,10 @@ SNK_API snk_status snk_build(int64_t M, int64_t K, int64_t nnz, int32_t* row, in
  * overwritten.  dt must equal the layout's dtype.  Asynchronous on `stream`.  Uses a
  * per-layout scratch region: calls of snk_forward on one layout must not overlap in time
  * (snk_backward_input has its own region and may overlap with snk_forward).
+ * For N >= 256 with X 16-byte aligned (base and ldx * element size) the product runs in the
+ * tensor-copy-staged wide kernel, whose shared-memory barrier waits are bounded (a wait
+ * that runs out is reported by snk_sync_status); other shapes take the nnz-balanced
+ * kernel.  The same holds for snk_backward_input with dY.
  */
 SNK_API snk_status snk_forward(const snk_layout* L, const void* values, const void* X, int64_t N, int64_t ldx,
                        void* Y, int64_t ldy, snk_dtype dt, snk_stream stream);

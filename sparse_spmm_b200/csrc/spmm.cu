@@ -22,8 +22,13 @@
 //
 // Gathered rows of the dense operand are kept packed (bf16 pairs in 32-bit words) until
 // the FMA and are multiplied with packed fp32 FMAs (two lanes of fp32 per instruction).
-// A lane holds up to 32 bytes of a row (two 16-byte vector loads), so few lanes repeat
-// the per-entry index and value loads.
+// A lane holds up to 32 bytes of a row (one 32-byte load where aligned), so few lanes
+// repeat the per-entry index and value loads.  Before waiting on the previous grid the
+// CTAs prefetch their share of every operand into L2.
+//
+// Wide dense operands (N >= 256) take a different kernel, k_spmm_tma: row blocks x
+// 128-column slices, the dense operand staged through shared memory by tensor-memory
+// copies in a warp-specialised producer/consumer pipeline (see its own comment).
 #include <algorithm>
 #include <type_traits>
 
