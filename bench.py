@@ -435,8 +435,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict:
     return out
 
 
-KERNEL_NAMES = {"forward": "k_spmm_small<bf16,*,*,false>", "backward_input": "k_spmm_small<bf16,*,*,true>",
-                "backward_weight": "k_sddmm_small<bf16,*,*>"}
+KERNEL_NAMES = {"forward": "k_spmm_small<bf16,*,*,false,int32_t>", "backward_input": "k_spmm_small<bf16,*,*,true,int32_t>",
+                "backward_weight": "k_sddmm_small<bf16,*,*,int32_t,false>"}
 
 
 def traffic_for(op: str):
