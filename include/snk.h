@@ -220,6 +220,21 @@ SNK_API snk_status snk_remap_entries(const int32_t* old_to_new, int64_t nnz, con
 SNK_API snk_status snk_set_index_bits(snk_layout* L, int32_t bits);
 
 /*
+ * snk_im2col3x3 -- the patch matrix of a 3x3 convolution (stride 1, zero padding 1, no
+ * bias), so that a sparse 3x3 layer is snk_forward with K = 9 C on it ("SparseRT", arXiv
+ * 2008.11849, Abstract: sparse 1x1 and 3x3 convolutions).  x: C x Nb x H x W, channel-major
+ * and contiguous, of dt.  out: (9 C) x (Nb H W) with leading dimension ld >= Nb H W:
+ * out[ci*9 + kh*3 + kw][(n*H + h)*W + w] = x[ci][n][h+kh-1][w+kw-1], or zero outside the
+ * image -- the column index of a [Co][C][3][3] weight flattened row-major.  Elements are
+ * copied bit for bit.  Asynchronous on `stream` (current device).  SNK_ERR_INVALID_ARG for
+ * sizes <= 0, 9 C > 65535, ld < Nb H W, null pointers or another dtype.  (The explicit
+ * patch matrix costs 9x the input in HBM traffic; the convolution oracle is the plain
+ * definition.)
+ */
+SNK_API snk_status snk_im2col3x3(const void* x, int64_t C, int64_t Nb, int64_t H, int64_t W, void* out, int64_t ld,
+                                 snk_dtype dt, snk_stream stream);
+
+/*
  * snk_sync_status -- synchronises `stream` and reports whether a product launch on this
  * layout gave up a bounded wait: the TMA-staged kernels for wide operands wait on
  * shared-memory barriers for the tensor copies, each wait for at most about a second.

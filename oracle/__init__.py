@@ -66,6 +66,10 @@ def _load():
         lib.orc_backward_weight.argtypes = [i64, vp, vp, vp, vp, i64, vp, vp]
         lib.orc_splitmix64.restype = None
         lib.orc_splitmix64.argtypes = [u64, i64, vp]
+        lib.orc_conv3x3.restype = None
+        lib.orc_conv3x3.argtypes = [i64, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp]
+        lib.orc_im2col3x3.restype = None
+        lib.orc_im2col3x3.argtypes = [i64, i64, i64, i64, ctypes.c_int, vp, vp, i64]
         lib.orc_restructure.restype = ctypes.c_int
         lib.orc_restructure.argtypes = [i64, i64, i64, vp, vp, vp, vp, ctypes.c_int, i64, u64, dbl,
                                         vp, vp, vp, vp, vp]
@@ -127,6 +131,24 @@ def build(M: int, K: int, row, col, values: np.ndarray, P: int) -> dict:
     if rc != 0:
         raise OracleError(rc)
     out["num_parts"] = int(peff[0])
+    return out
+
+
+def conv3x3(Co: int, C: int, Nb: int, H: int, W: int, row, col, vals64, X64) -> tuple[np.ndarray, np.ndarray]:
+    """3x3 convolution, stride 1, zero padding 1, of X (C x Nb x H x W) by the sparse kernel
+    given as entries (co, ci*9 + kh*3 + kw); returns (Y, A), Co x (Nb*H*W) float64."""
+    row, col = _c(row, np.int32), _c(col, np.int32)
+    v, X = _c(vals64, np.float64), _c(np.asarray(X64).reshape(C, Nb * H * W), np.float64)
+    Y = np.empty((Co, Nb * H * W)); A = np.empty((Co, Nb * H * W))
+    _load().orc_conv3x3(Co, C, Nb, H, W, row.size, _p(row), _p(col), _p(v), _p(X), _p(Y), _p(A))
+    return Y, A
+
+
+def im2col3x3(C: int, Nb: int, H: int, W: int, X: np.ndarray) -> np.ndarray:
+    """Patch matrix (9C) x (Nb*H*W) of X (C x Nb x H x W; float32 or bf16 bits), bit for bit."""
+    X = np.ascontiguousarray(X)
+    out = np.empty((9 * C, Nb * H * W), dtype=X.dtype)
+    _load().orc_im2col3x3(C, Nb, H, W, X.itemsize, _p(X), _p(out), Nb * H * W)
     return out
 
 

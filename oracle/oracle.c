@@ -20,6 +20,11 @@
  *                    O7: dW[e]   = sum over n of dY[row_e, n] * X[col_e, n]
  *   orc_restructure  O8: magnitude drop of k entries, random regrowth of k positions drawn
  *                    from a SplitMix64 stream, rebuild of the sorted COO.
+ *   orc_conv3x3      a 3x3 convolution (stride 1, zero padding 1, no bias) of a
+ *                    channel-major input by a sparse kernel whose column index is
+ *                    ci*9 + kh*3 + kw ("SparseRT", arXiv 2008.11849, Abstract: sparse
+ *                    1x1 and 3x3 convolutions), straight from the definition.
+ *   orc_im2col3x3    the patch matrix of that convolution, element bits copied.
  *
  * Every product is accumulated in double.  Each fp routine also returns, per output,
  * the sum of absolute values of its terms (A), which scales the parity tolerance.
@@ -345,4 +350,54 @@ int orc_restructure(int64_t M, int64_t K, int64_t nnz, const int32_t* row, const
   free(dropped);
   free(it);
   return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 3x3 convolution */
+
+/* Y[co][n][h][w] = sum over entries (co, c = ci*9 + kh*3 + kw) of v * X[ci][n][h+kh-1][w+kw-1],
+ * terms outside the image being zero.  X: C x Nb x H x W, Y: Co x Nb x H x W, row-major. */
+void orc_conv3x3(int64_t Co, int64_t C, int64_t Nb, int64_t H, int64_t W, int64_t nnz, const int32_t* row,
+                 const int32_t* col, const double* val, const double* X, double* Y, double* A) {
+  (void)C;
+  const int64_t P = Nb * H * W;
+  for (int64_t i = 0; i < Co * P; ++i) {
+    Y[i] = 0.0;
+    A[i] = 0.0;
+  }
+  for (int64_t e = 0; e < nnz; ++e) {
+    const int64_t co = row[e], ci = col[e] / 9, kh = (col[e] / 3) % 3, kw = col[e] % 3;
+    for (int64_t n = 0; n < Nb; ++n)
+      for (int64_t h = 0; h < H; ++h)
+        for (int64_t w = 0; w < W; ++w) {
+          const int64_t hs = h + kh - 1, ws = w + kw - 1;
+          if (hs < 0 || hs >= H || ws < 0 || ws >= W) continue;
+          const double t = val[e] * X[((ci * Nb + n) * H + hs) * W + ws];
+          Y[co * P + (n * H + h) * W + w] += t;
+          A[co * P + (n * H + h) * W + w] += fabs(t);
+        }
+  }
+}
+
+/* Patch matrix of the convolution above: out[(ci*9 + kh*3 + kw)][(n*H + h)*W + w] =
+ * X[ci][n][h+kh-1][w+kw-1], or all-zero bits outside the image.  Elements of `elem`
+ * bytes are copied bit for bit; out has row stride ld (elements). */
+void orc_im2col3x3(int64_t C, int64_t Nb, int64_t H, int64_t W, int elem, const void* X, void* out, int64_t ld) {
+  const int64_t P = Nb * H * W;
+  const unsigned char* x = (const unsigned char*)X;
+  unsigned char* o = (unsigned char*)out;
+  for (int64_t ci = 0; ci < C; ++ci)
+    for (int64_t k = 0; k < 9; ++k) {
+      const int64_t kh = k / 3, kw = k % 3, r = ci * 9 + k;
+      for (int64_t n = 0; n < Nb; ++n)
+        for (int64_t h = 0; h < H; ++h)
+          for (int64_t w = 0; w < W; ++w) {
+            const int64_t hs = h + kh - 1, ws = w + kw - 1, j = (n * H + h) * W + w;
+            unsigned char* dst = o + (r * ld + j) * elem;
+            if (hs < 0 || hs >= H || ws < 0 || ws >= W)
+              memset(dst, 0, (size_t)elem);
+            else
+              memcpy(dst, x + (((ci * Nb + n) * H + hs) * W + ws) * elem, (size_t)elem);
+          }
+    }
+  (void)P;
 }

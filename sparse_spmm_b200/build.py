@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libsnk.so")
-SOURCES = ["snk.cu", "format.cu", "spmm.cu", "noalloc.cu", "probe.cu"]
+SOURCES = ["snk.cu", "format.cu", "spmm.cu", "noalloc.cu", "probe.cu", "conv.cu"]
 HEADERS = ["internal.cuh"]
 
 NVCC_FLAGS = [

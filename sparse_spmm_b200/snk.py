@@ -179,6 +179,29 @@ def snk_csr_forward_static(M, K, row_ptr, col, values, X, Y, num_parts=0, stream
               _ld(X), _ptr(Y), _ld(Y), num_parts, _stream(stream)), "snk_csr_forward_static")
 
 
+def snk_im2col3x3(x, C, Nb, H, W, out=None, stream=None):
+    """Patch matrix (9C) x (Nb*H*W) of a channel-major x (C x Nb x H x W) for a 3x3 convolution."""
+    lib = load_library()
+    lib.snk_im2col3x3.restype = ctypes.c_int
+    lib.snk_im2col3x3.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous (C x Nb x H x W)")
+    if out is None:
+        out = torch.empty((9 * C, Nb * H * W), dtype=x.dtype, device=x.device)
+    _check(lib.snk_im2col3x3(_ptr(x), C, Nb, H, W, _ptr(out), _ld(out), _dtype_code(x.dtype), _stream(stream)),
+           "snk_im2col3x3")
+    return out
+
+
+def sparse_conv3x3(L, x, Nb, H, W, patch=None, Y=None, stream=None):
+    """A sparse 3x3 convolution (stride 1, padding 1): Y (Co x Nb*H*W) = W * x with W held by
+    layout L (Co x 9C, column ci*9 + kh*3 + kw) and x channel-major (C x Nb x H x W)."""
+    C = L.K // 9
+    patch = snk_im2col3x3(x, C, Nb, H, W, out=patch, stream=stream)
+    return L.forward(patch, Y=Y, stream=stream)
+
+
 def snk_remap_entries(old_to_new, src, dst, stream=None):
     """dst[old_to_new[e]] = src[e] for surviving entries, 0 elsewhere (state across a restructure)."""
     lib = load_library()
