@@ -746,6 +746,41 @@ def run_sweep(args) -> None:
             del copies
             torch.cuda.empty_cache()
 
+    # sparse 3x3 convolutions at ResNet-50 layer shapes (channel-major input, batch 32):
+    # patch matrix + forward SpMM, against cuDNN's dense fp32 convolution (TF32 off)
+    torch.backends.cudnn.allow_tf32 = False
+    for (Cc, HW, sp) in ((256, 14, 0.90), (256, 14, 0.95), (512, 7, 0.90), (512, 7, 0.95)):
+        Nb, H, W = 32, HW, HW
+        P = Nb * H * W
+        layer = wl.uniform_layer(Cc, 9 * Cc, sp, "f32", args.seed, "W3x3")
+        xin = np.maximum(np.random.default_rng(args.seed).normal(size=(Cc, P)), 0).astype(np.float32)
+        hot = layer.nnz * 8 + Cc * P * 4 * 11  # W, input, patch matrix (9x), output
+        R = int(min(20, max(2, np.ceil(3 * l2 / hot))))
+        Ls = [snk.Layout(Cc, 9 * Cc, dev_t(layer.row), dev_t(layer.col), dev_t(layer.values)) for _ in range(R)]
+        xs = [dev_t(xin) for _ in range(R)]
+        patches = [torch.empty((9 * Cc, P), device="cuda") for _ in range(R)]
+        ys = [torch.empty((Cc, P), device="cuda") for _ in range(R)]
+        fns = [lambda i=i: snk.sparse_conv3x3(Ls[i], xs[i], Nb, H, W, patch=patches[i], Y=ys[i]) for i in range(R)]
+        us = _graph_time_us(fns, reps=5)
+        im2 = [lambda i=i: snk.snk_im2col3x3(xs[i], Cc, Nb, H, W, out=patches[i]) for i in range(R)]
+        us_patch = _graph_time_us(im2, reps=5)
+        Wd = torch.zeros(Cc, 9 * Cc, device="cuda")
+        Wd[dev_t(layer.row).long(), dev_t(layer.col).long()] = dev_t(layer.values)
+        Wd4 = Wd.view(Cc, Cc, 3, 3)
+        xn = [x.view(Cc, Nb, H, W).permute(1, 0, 2, 3).contiguous() for x in xs]  # NCHW for cuDNN
+        dense = [lambda i=i: torch.nn.functional.conv2d(xn[i], Wd4, padding=1) for i in range(R)]
+        us_dense = _graph_time_us(dense, reps=5)
+        fl = op_flops(layer.nnz, P)
+        b = layer.nnz * 8 + 4 * (Cc + 1) + Cc * P * 4 * 2  # W once, input once, output once
+        print(json.dumps({"sweep": f"conv3x3-{Cc}x{Cc}-{H}x{W}-b32-s{int(round(sp * 100))}-f32", "layer": "W3x3",
+                          "M": Cc, "K": 9 * Cc, "nnz": layer.nnz, "op": "conv3x3", "N": P, "us": round(us, 2),
+                          "patch_us": round(us_patch, 2), "gbs_implicit_model": round(b / us / 1e3, 1),
+                          "gflops": round(fl / us / 1e3, 1), "frac_fp32": round(fl / us / 1e6 / f32["tflops"], 4),
+                          "dense_cudnn_fp32_us": round(us_dense, 2), "speedup_vs_dense": round(us_dense / us, 2)}),
+              flush=True)
+        del Ls, xs, patches, ys, xn, Wd, Wd4
+        torch.cuda.empty_cache()
+
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
