@@ -1144,17 +1144,18 @@ template <typename T, bool TRANS, typename I>
 using SpmmKernel = void (*)(const SpmmArgs<T, I>);
 
 // Instantiated shapes: 32-byte groups (NC = 16 bf16 / 8 fp32) with G = 1..64/NC lanes,
-// 16-, 8- and 4-byte groups with one lane, and scalars with G = 1..32.
+// 16-byte groups with one or two lanes (two when a 32-byte operand row is split between
+// them), 8- and 4-byte groups with one lane, and scalars with G = 1..32.
 template <typename T, bool TRANS, typename I>
 SpmmKernel<T, TRANS, I> pick_spmm(int nc, int g) {
 #define SNK_CASE(NC_, G_) \
   if (nc == NC_ && g == G_) return k_spmm_small<T, NC_, G_, TRANS, I>;
   if constexpr (sizeof(T) == 2) {
     SNK_CASE(16, 1) SNK_CASE(16, 2) SNK_CASE(16, 4)
-    SNK_CASE(8, 1) SNK_CASE(4, 1) SNK_CASE(2, 1)
+    SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(4, 1) SNK_CASE(2, 1)
   } else {
     SNK_CASE(8, 1) SNK_CASE(8, 2) SNK_CASE(8, 4) SNK_CASE(8, 8)
-    SNK_CASE(4, 1) SNK_CASE(2, 1)
+    SNK_CASE(4, 1) SNK_CASE(4, 2) SNK_CASE(2, 1)
   }
   SNK_CASE(1, 1) SNK_CASE(1, 2) SNK_CASE(1, 4) SNK_CASE(1, 8) SNK_CASE(1, 16) SNK_CASE(1, 32)
 #undef SNK_CASE
@@ -1277,6 +1278,10 @@ snk_status spmm_typed(const snk_layout* L, const I* idx, const T* values, const 
       g = pow2ceil(ncols);
     }
     g = std::min(g, 32);
+    if (g == 1 && nc * elem == 32) {  // a one-lane worker of 32 bytes: two lanes of 16 (measured faster)
+      nc /= 2;
+      g = 2;
+    }
     const int nt = nc * g;
     const int tiles = (ncols + nt - 1) / nt;
     auto kern = pick_spmm<T, TRANS, I>(nc, g);
