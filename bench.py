@@ -553,10 +553,22 @@ def run_profile(args) -> None:
     if args.profile_workload == "gpt2-w1":  # GPT-2 c_fc, 3072 x 768 at 90% (magnitude-pruned), fp32, N = 1024
         layer = wl.magnitude_pruned_layer(3072, 768, 0.90, args.seed, "W1")
         batches = [1024]
+    elif args.profile_workload == "gpt2-w2":  # GPT-2 c_proj, 768 x 3072 at 90%, fp32, N = 1024
+        layer = wl.magnitude_pruned_layer(768, 3072, 0.90, args.seed + 1, "W2")
+        batches = [1024]
     elif args.profile_workload == "conv-512x2048-s80":  # 1x1 conv, fp32, N = 6272, X = ReLU(N(0,1))
         layer = wl.uniform_layer(512, 2048, 0.80, "f32", args.seed, "W")
         batches = [6272]
         relu = True
+    elif args.profile_workload == "tiny-fc":  # 512 x 512 at 90%, fp32, N = 8
+        layer = wl.uniform_layer(512, 512, 0.90, "f32", args.seed, "W")
+        batches = [8]
+    elif args.profile_workload == "llama-up":  # 11008 x 4096 at 99%, Zipf(1.2) rows, bf16, N = 1, 4, 16
+        layer = wl.zipf_layer(11008, 4096, 0.99, "bf16", 1.2, args.seed, "W_up")
+        batches = [1, 4, 16]
+    elif args.profile_workload == "llama-down":  # 4096 x 11008 at 99%, Zipf(1.2) rows, bf16, N = 1, 4, 16
+        layer = wl.zipf_layer(4096, 11008, 0.99, "bf16", 1.2, args.seed + 1, "W_down")
+        batches = [1, 4, 16]
     else:  # the bench workload
         layer = wl.uniform_layer(4096, 4096, 0.95, "bf16", seed=args.seed, name="W")
         batches = [int(b) for b in args.batches.split(",")]
@@ -796,8 +808,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run two untimed passes of the step (for ncu captures) and exit")
-    ap.add_argument("--profile-workload", default="fc", choices=("fc", "gpt2-w1", "conv-512x2048-s80"),
-                    help="workload of --profile: the bench's FC layer, GPT-2 c_fc at N=1024, or a 1x1 conv at N=6272")
+    ap.add_argument("--profile-workload", default="fc",
+                    choices=("fc", "gpt2-w1", "gpt2-w2", "conv-512x2048-s80", "tiny-fc", "llama-up", "llama-down"),
+                    help="workload of --profile: the bench's FC layer or another config's layer")
     ap.add_argument("--sweep", action="store_true",
                     help="time every config, op and batch (plus dense baselines); JSON lines; exit")
     args = ap.parse_args()
